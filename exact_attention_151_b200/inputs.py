@@ -1,0 +1,104 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the smoke check.
+
+This module only draws random numbers; it holds none of the attention
+arithmetic. Both the CUDA path and the CPU oracle receive the exact 16-bit
+tensors made here (the oracle as raw bit patterns).
+
+Recipe: torch's CPU generator seeded with ``seed``; Q, K and V are drawn in
+that order, each as float32 in [B, N, H, D] layout, scaled / shifted to the
+workload's distribution and then rounded to the 16-bit dtype on the host.
+The pages fix no generator, so this one is a stated choice.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention-forward problem: sizes, dtype, mask and input distributions."""
+
+    name: str
+    B: int
+    N: int
+    H: int
+    D: int
+    dtype: str = "bf16"
+    causal: bool = False
+    q_std: float = 1.0
+    k_std: float = 1.0
+    v_dist: str = "normal"  # "normal" (N(0,1)) or "uniform" (U(-1, 1))
+    seed: int = 0
+    scale: float | None = None  # None means 1/sqrt(D)
+    notes: dict = field(default_factory=dict, compare=False)
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.D)
+
+    @property
+    def flops(self) -> float:
+        """4*B*H*N^2*D, halved when causal (the metric's counting convention)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.D
+        return f / 2 if self.causal else f
+
+    @property
+    def min_hbm_bytes(self) -> int:
+        """Read Q, K, V once, write O once (16-bit) and LSE (fp32)."""
+        return 8 * self.B * self.N * self.H * self.D + 4 * self.B * self.H * self.N
+
+    def with_(self, **kw) -> "Workload":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return Workload(**d)
+
+
+def _sweep(n: int, causal: bool) -> Workload:
+    tag = "causal" if causal else "noncausal"
+    return Workload(f"sweep_n{n}_{tag}", B=32768 // n, N=n, H=16, D=128, causal=causal)
+
+
+# The five published configurations, named by what they are.
+WORKLOADS: dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("small_b1h2n256d64", B=1, N=256, H=2, D=64),
+        Workload("llama7b_b4h32n2048d128_causal", B=4, N=2048, H=32, D=128, causal=True),
+        Workload("long_b1h32n8192d128_noncausal", B=1, N=8192, H=32, D=128),
+        Workload("long_b1h32n8192d128_causal", B=1, N=8192, H=32, D=128, causal=True),
+        *[_sweep(n, c) for c in (False, True) for n in (1024, 4096, 16384, 32768)],
+        Workload("stress_b2h16n4093d64_fp16_causal", B=2, N=4093, H=16, D=64, dtype="fp16", causal=True,
+                 q_std=4.0, v_dist="uniform"),
+        # Supplementary: Q ~ N(0, 16^2) so that logits really reach ~100 (the
+        # stated regime); the configuration as written peaks near 25-30.
+        Workload("stress_hot_b2h16n4093d64_fp16_causal", B=2, N=4093, H=16, D=64, dtype="fp16", causal=True,
+                 q_std=16.0, v_dist="uniform"),
+    ]
+}
+
+
+def make_qkv(w: Workload, seed: int | None = None):
+    """Return (q, k, v) as contiguous CPU tensors of w.dtype in [B, N, H, D]."""
+    g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    shape = (w.B, w.N, w.H, w.D)
+    q = torch.randn(shape, generator=g, dtype=torch.float32) * w.q_std
+    k = torch.randn(shape, generator=g, dtype=torch.float32) * w.k_std
+    if w.v_dist == "uniform":
+        v = torch.rand(shape, generator=g, dtype=torch.float32) * 2.0 - 1.0
+    else:
+        v = torch.randn(shape, generator=g, dtype=torch.float32)
+    dt = TORCH_DTYPES[w.dtype]
+    return q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous()
+
+
+def bits(t: torch.Tensor):
+    """Raw 16-bit patterns of a CPU bf16/fp16 tensor as a numpy uint16 array."""
+    import numpy as np
+
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -1,0 +1,303 @@
+// Test infrastructure, not product code.
+//
+// Plain, slow, fp64 reference for the exact attention forward that the CUDA
+// library computes. Only the test suite, the smoke check and the bench's
+// CPU-baseline leg may load this library; the product path never does.
+//
+// What it computes (the plain definition, written out):
+//   * "Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V" and its four steps
+//     (similarity, scaling, softmax, weighted sum of V): llmtrend.com,
+//     "FlashAttention: ...", section on the self-attention bottleneck.
+//   * the same computation written as matmul / divide / softmax / matmul on
+//     [batch, heads, seq, seq] scores: the tuning handbook chapter 3
+//     ("MHA performance tuning"), section "where the MHA memory bottleneck is".
+//   * causal attention skips future key positions: same chapter, section
+//     "practical notes" (causal mask bullet).
+//   * max subtraction before exp (the log-sum-exp trick) and a per-row
+//     log-sum-exp: llmtrend.com page, "numerical stability" bullet; the
+//     handbook's tiled routine keeps lse[B,H,N] and updates it with log().
+//
+// For each (b, h, i), with vis(i) = { j : 0 <= j < N and (j <= i if causal) }:
+//   s_j   = scale * sum_d q[b,i,h,d] * k[b,j,h,d]      (d ascending)
+//   m     = max_{j in vis} s_j
+//   l     = sum_{j in vis} exp(s_j - m)                  (j ascending)
+//   O_d   = (sum_{j in vis} exp(s_j - m) * v[b,j,h,d]) / l
+//   LSE   = m + log(l)                                    (natural log)
+//
+// Inputs are the raw 16-bit patterns (bf16 or fp16) of Q, K, V in
+// [B, N, H, D] order; they are widened to double exactly. Outputs are double:
+// O in [B, N, H, D], LSE in [B, H, N].
+//
+// A second, algorithmically different statement is also here: the tiled
+// online-softmax routine printed in the handbook chapter (section "engineering
+// implementation"), restated in fp64 with two readings: the block max is taken
+// with keepdim (the printed code mixes a [B,H,bs] lse slice with a
+// [B,H,bs,1] max), and the routine returns its lse as well as its output.
+// Its algebra is exact, so it must agree with the plain definition to
+// rounding; the tests use that as an independent pin.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits.
+double decode_fp16(uint16_t h) {
+  const int sign = (h >> 15) & 1;
+  const int e = (h >> 10) & 0x1f;
+  const int f = h & 0x3ff;
+  double mag;
+  if (e == 0) {
+    mag = std::ldexp(static_cast<double>(f), -24);  // subnormal: f * 2^-24
+  } else if (e == 31) {
+    mag = f ? std::numeric_limits<double>::quiet_NaN()
+            : std::numeric_limits<double>::infinity();
+  } else {
+    mag = std::ldexp(static_cast<double>(1024 + f), e - 25);  // (1.f) * 2^(e-15)
+  }
+  return sign ? -mag : mag;
+}
+
+// bfloat16: 1 sign, 8 exponent (bias 127), 7 fraction bits.
+double decode_bf16(uint16_t h) {
+  const int sign = (h >> 15) & 1;
+  const int e = (h >> 7) & 0xff;
+  const int f = h & 0x7f;
+  double mag;
+  if (e == 0) {
+    mag = std::ldexp(static_cast<double>(f), -133);  // subnormal: f * 2^-133
+  } else if (e == 255) {
+    mag = f ? std::numeric_limits<double>::quiet_NaN()
+            : std::numeric_limits<double>::infinity();
+  } else {
+    mag = std::ldexp(static_cast<double>(128 + f), e - 134);  // (1.f) * 2^(e-127)
+  }
+  return sign ? -mag : mag;
+}
+
+double decode(uint16_t h, int dtype) { return dtype == 0 ? decode_bf16(h) : decode_fp16(h); }
+
+struct Problem {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t B, N, H, D;
+  double scale;
+  int causal;
+  int dtype;
+};
+
+// Index of element (b, n, h, d) in a contiguous [B, N, H, D] tensor.
+inline int64_t at(const Problem& p, int64_t b, int64_t n, int64_t h, int64_t d) {
+  return ((b * p.N + n) * p.H + h) * p.D + d;
+}
+
+// Widen the (b, h) head of a [B,N,H,D] tensor to a dense [N][D] double block.
+void widen_head(const Problem& p, const uint16_t* src, int64_t b, int64_t h, std::vector<double>& dst) {
+  dst.resize(static_cast<size_t>(p.N * p.D));
+  for (int64_t n = 0; n < p.N; ++n)
+    for (int64_t d = 0; d < p.D; ++d) dst[n * p.D + d] = decode(src[at(p, b, n, h, d)], p.dtype);
+}
+
+int64_t visible_count(const Problem& p, int64_t i) { return p.causal ? (i + 1) : p.N; }
+
+// One query row of the definition, given that row's materialised scores
+// s[0 .. nvis-1]. Writes O[0..D-1] and returns LSE.
+double finish_row(const Problem& p, const double* s, int64_t nvis, const std::vector<double>& V,
+                  double* o_out) {
+  double m = -std::numeric_limits<double>::infinity();
+  for (int64_t j = 0; j < nvis; ++j) m = s[j] > m ? s[j] : m;
+  double l = 0.0;
+  for (int64_t j = 0; j < nvis; ++j) l += std::exp(s[j] - m);
+  for (int64_t d = 0; d < p.D; ++d) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < nvis; ++j) acc += std::exp(s[j] - m) * V[j * p.D + d];
+    o_out[d] = acc / l;
+  }
+  return m + std::log(l);
+}
+
+// s_j for one query row i against all keys j < nvis.
+void score_row(const Problem& p, const std::vector<double>& Q, const std::vector<double>& K, int64_t i,
+               int64_t nvis, double* s) {
+  const double* qi = &Q[i * p.D];
+  for (int64_t j = 0; j < nvis; ++j) {
+    const double* kj = &K[j * p.D];
+    double dot = 0.0;
+    for (int64_t d = 0; d < p.D; ++d) dot += qi[d] * kj[d];
+    s[j] = p.scale * dot;
+  }
+}
+
+template <class F>
+void parallel_for(int64_t n, int nthreads, F&& fn) {
+  if (nthreads <= 1 || n <= 1) {
+    fn(0, n);
+    return;
+  }
+  const int64_t nt = nthreads < n ? nthreads : n;
+  std::vector<std::thread> pool;
+  for (int64_t t = 0; t < nt; ++t) {
+    const int64_t lo = n * t / nt, hi = n * (t + 1) / nt;
+    pool.emplace_back([&fn, lo, hi] { fn(lo, hi); });
+  }
+  for (auto& th : pool) th.join();
+}
+
+bool valid(const Problem& p) {
+  return p.q && p.k && p.v && p.B >= 0 && p.N >= 0 && p.H >= 0 && p.D >= 1 && (p.dtype == 0 || p.dtype == 1);
+}
+
+}  // namespace
+
+extern "C" {
+
+// Widen n 16-bit patterns to double (dtype 0 = bf16, 1 = fp16).
+int oracle_decode16(const uint16_t* src, int64_t n, int dtype, double* dst) {
+  if (!src || !dst || n < 0 || (dtype != 0 && dtype != 1)) return 1;
+  for (int64_t i = 0; i < n; ++i) dst[i] = decode(src[i], dtype);
+  return 0;
+}
+
+// The definition with the whole N x N score matrix of one (b, h) materialised
+// in memory (rows filled by `nthreads` threads). O: [B,N,H,D], LSE: [B,H,N].
+int oracle_attention_full(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B, int64_t N,
+                          int64_t H, int64_t D, double scale, int causal, int dtype, double* o, double* lse,
+                          int nthreads) {
+  Problem p{q, k, v, B, N, H, D, scale, causal, dtype};
+  if (!valid(p) || !o || !lse) return 1;
+  std::vector<double> Q, K, V;
+  std::vector<double> S(static_cast<size_t>(N) * static_cast<size_t>(N));
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t h = 0; h < H; ++h) {
+      widen_head(p, q, b, h, Q);
+      widen_head(p, k, b, h, K);
+      widen_head(p, v, b, h, V);
+      parallel_for(N, nthreads, [&](int64_t lo, int64_t hi) {
+        for (int64_t i = lo; i < hi; ++i) score_row(p, Q, K, i, visible_count(p, i), &S[i * N]);
+      });
+      parallel_for(N, nthreads, [&](int64_t lo, int64_t hi) {
+        std::vector<double> orow(static_cast<size_t>(D));
+        for (int64_t i = lo; i < hi; ++i) {
+          const double L = finish_row(p, &S[i * N], visible_count(p, i), V, orow.data());
+          for (int64_t d = 0; d < D; ++d) o[at(p, b, i, h, d)] = orow[d];
+          lse[(b * H + h) * N + i] = L;
+        }
+      });
+    }
+  }
+  return 0;
+}
+
+// The same definition for a list of (b, h, i) triples, one score row at a
+// time. rows: [nrows][3]; o_rows: [nrows][D]; lse_rows: [nrows]. Rows are
+// independent, so this is bit-identical to oracle_attention_full on them.
+int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B, int64_t N,
+                          int64_t H, int64_t D, double scale, int causal, int dtype, const int64_t* rows,
+                          int64_t nrows, double* o_rows, double* lse_rows, int nthreads) {
+  Problem p{q, k, v, B, N, H, D, scale, causal, dtype};
+  if (!valid(p) || !rows || nrows < 0 || (nrows > 0 && (!o_rows || !lse_rows))) return 1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= N) return 2;
+  }
+  parallel_for(nrows, nthreads, [&](int64_t lo, int64_t hi) {
+    std::vector<double> qrow(static_cast<size_t>(D)), krow(static_cast<size_t>(D));
+    std::vector<double> s, Vvis;
+    for (int64_t r = lo; r < hi; ++r) {
+      const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+      const int64_t nvis = visible_count(p, i);
+      s.assign(static_cast<size_t>(nvis), 0.0);
+      Vvis.assign(static_cast<size_t>(nvis * D), 0.0);
+      for (int64_t d = 0; d < D; ++d) qrow[d] = decode(q[at(p, b, i, h, d)], dtype);
+      for (int64_t j = 0; j < nvis; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qrow[d] * decode(k[at(p, b, j, h, d)], dtype);
+        s[j] = scale * dot;
+        for (int64_t d = 0; d < D; ++d) Vvis[j * D + d] = decode(v[at(p, b, j, h, d)], dtype);
+      }
+      lse_rows[r] = finish_row(p, s.data(), nvis, Vvis, &o_rows[r * D]);
+    }
+  });
+  return 0;
+}
+
+// The handbook's tiled online-softmax routine, in fp64, one (b, h) at a time.
+// For every query block [qs, qe) and every key block [ks, ke) (both cut at
+// block_size, the last one truncated at N):
+//   scores    = scale * Q_blk K_blk^T            (future keys = -inf if causal)
+//   blk_max   = row max of scores                (keepdim reading)
+//   mu        = max(lse, blk_max)
+//   e_new     = exp(scores - mu),  e_old = exp(lse - mu)
+//   out       = (out * e_old + e_new V_blk) / (e_old + rowsum(e_new))
+//   lse       = mu + log(e_old + rowsum(e_new))
+// Key blocks that lie wholly in the future of every row of the query block
+// are skipped (the causal reading); key block 0 always holds a visible key,
+// so lse is finite after it and mu never subtracts -inf from -inf.
+int oracle_tiled_reference(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B, int64_t N,
+                           int64_t H, int64_t D, double scale, int causal, int dtype, int64_t block_size,
+                           double* o, double* lse) {
+  Problem p{q, k, v, B, N, H, D, scale, causal, dtype};
+  if (!valid(p) || !o || !lse || block_size < 1) return 1;
+  const double ninf = -std::numeric_limits<double>::infinity();
+  std::vector<double> Q, K, V;
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t h = 0; h < H; ++h) {
+      widen_head(p, q, b, h, Q);
+      widen_head(p, k, b, h, K);
+      widen_head(p, v, b, h, V);
+      for (int64_t qs = 0; qs < N; qs += block_size) {
+        const int64_t qe = qs + block_size < N ? qs + block_size : N;
+        const int64_t nq = qe - qs;
+        std::vector<double> out(static_cast<size_t>(nq * D), 0.0);
+        std::vector<double> run_lse(static_cast<size_t>(nq), ninf);
+        for (int64_t ks = 0; ks < N; ks += block_size) {
+          if (causal && ks > qe - 1) break;  // every key of this block is in every row's future
+          const int64_t ke = ks + block_size < N ? ks + block_size : N;
+          const int64_t nk = ke - ks;
+          for (int64_t r = 0; r < nq; ++r) {
+            const int64_t i = qs + r;
+            std::vector<double> sc(static_cast<size_t>(nk));
+            double bmax = ninf;
+            for (int64_t c = 0; c < nk; ++c) {
+              const int64_t j = ks + c;
+              if (causal && j > i) {
+                sc[c] = ninf;
+              } else {
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d) dot += Q[i * D + d] * K[j * D + d];
+                sc[c] = scale * dot;
+              }
+              bmax = sc[c] > bmax ? sc[c] : bmax;
+            }
+            const double mu = run_lse[r] > bmax ? run_lse[r] : bmax;
+            const double e_old = std::exp(run_lse[r] - mu);
+            double e_sum = 0.0;
+            std::vector<double> e(static_cast<size_t>(nk));
+            for (int64_t c = 0; c < nk; ++c) {
+              e[c] = std::exp(sc[c] - mu);
+              e_sum += e[c];
+            }
+            for (int64_t d = 0; d < D; ++d) {
+              double pv = 0.0;
+              for (int64_t c = 0; c < nk; ++c) pv += e[c] * V[(ks + c) * D + d];
+              out[r * D + d] = (out[r * D + d] * e_old + pv) / (e_old + e_sum);
+            }
+            run_lse[r] = mu + std::log(e_old + e_sum);
+          }
+        }
+        for (int64_t r = 0; r < nq; ++r) {
+          for (int64_t d = 0; d < D; ++d) o[at(p, b, qs + r, h, d)] = out[r * D + d];
+          lse[(b * H + h) * N + qs + r] = run_lse[r];
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+}  // extern "C"
