@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of the fused exact-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one fa_fwd call over the whole workload (default: the Llama-7B-shaped
+causal forward, B=4 H=32 N=2048 D=128 bf16). Prints ONE JSON line on rank 0.
+
+  value      forward TFLOP/s of the whole job (4*B*H*N^2*D per step, halved for
+             causal) with inputs resident in HBM; device time from CUDA events
+             around exactly K steps (barrier + synchronize on both sides), max
+             over ranks. Q+K+V+O (256 MiB at the default) exceed the 126 MB L2,
+             so no flush is done between steps.
+  e2e        the same metric through the public API with pinned host buffers:
+             each step copies Q, K, V host->device, runs fa_fwd and copies O and
+             LSE back, all inside the timed region.
+  roofline   tensor-core bound: achieved TFLOP/s of the kernel against the
+             measured cuBLAS bf16 peak; dram traffic per launch from the
+             committed ncu summary when it matches the current kernel source.
+  cpu_baseline  the fp64 oracle on a bounded row sample, on the host cores
+             (rank 0 at N=1 only); the same rows double as a parity check.
+
+With torchrun (N>1) every rank runs the full workload on its own GPU (weak
+scaling, no collective on the data path); the timing is reduced with MAX.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
+DEFAULT_WORKLOAD = "llama7b_b4h32n2048d128_causal"
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_151_b200", "csrc", f) for f in ("fa_fwd.cu", "sm100.cuh")]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAK_TFLOPS = 1590.0
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"]), e.get("how", "")
+    except Exception:
+        pass
+    return None, None
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, throttle reasons) in a thread during the timed region."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+        0x0000000000000002: "applications_clocks_setting",
+    }
+
+    def __init__(self, uuid: str, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(u.encode() if isinstance(u, str) else u)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self._nvml = None
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+             "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+        if self.error:
+            d["error"] = self.error
+        return d
+
+
+def row_flops(w, rows) -> float:
+    """Algorithmic flops of the sampled rows: 4*D per visible key (QK^T and PV)."""
+    import numpy as np
+
+    rows = np.asarray(rows)
+    nvis = (rows[:, 2] + 1) if w.causal else np.full(len(rows), w.N)
+    return float(4.0 * w.D * nvis.sum())
+
+
+def oracle_row_sample(w, q, k, v, target_s: float, seed: int = 0):
+    """Time the oracle on a row sample sized to roughly target_s seconds of host work."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_151_b200.inputs import bits
+
+    Q, K, V = bits(q), bits(k), bits(v)
+    rng = np.random.default_rng(seed)
+    threads = oracle.default_threads()
+
+    def draw(n):
+        return np.stack([rng.integers(0, w.B, n), rng.integers(0, w.H, n), rng.integers(0, w.N, n)], axis=1)
+
+    probe = draw(max(threads, 8))
+    t0 = time.perf_counter()
+    oracle.attention_rows(Q, K, V, w.softmax_scale, w.causal, w.dtype, probe, nthreads=threads)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n = int(max(threads, min(200000, len(probe) * target_s / dt)))
+    rows = draw(n)
+    t0 = time.perf_counter()
+    o_ref, lse_ref = oracle.attention_rows(Q, K, V, w.softmax_scale, w.causal, w.dtype, rows, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return rows, o_ref, lse_ref, dt, threads
+
+
+def run_reference(args, w):
+    """The oracle on the host cores, each step a bounded row sample (rank 0 only)."""
+    import numpy as np
+
+    from exact_attention_151_b200.inputs import make_qkv
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v = make_qkv(w)
+    per_step_target = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        rows, _, _, dt, threads = oracle_row_sample(w, q, k, v, per_step_target, seed=100 + i)
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(row_flops(w, rows))
+    value = sum(flops) / sum(times) / 1e12
+    sample = (f"{len(rows)} random (b,h,i) rows per step of the {w.name} workload "
+              f"(~{per_step_target:.0f} s of fp64 work per step)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "dtype": w.dtype, "causal": w.causal,
+            "scale": w.softmax_scale, "flops_per_step": w.flops, "seed": w.seed,
+            "inputs": f"Q~N(0,{w.q_std}^2) K~N(0,{w.k_std}^2) V~{'U(-1,1)' if w.v_dist == 'uniform' else 'N(0,1)'}",
+            "l2": "no flush: Q+K+V+O exceed the 126 MB L2" if 8 * w.B * w.N * w.H * w.D > 126e6 else
+                  "L2 flushed between steps (256 MiB write, outside the per-step kernel events)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from exact_attention_151_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_151_b200 as fa
+    from exact_attention_151_b200.inputs import make_qkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    q, k, v = make_qkv(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flush = None
+    if 8 * w.B * w.N * w.H * w.D <= 126e6:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
+
+    for _ in range(args.warmup):
+        step()
+    if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
+        raise RuntimeError("device status word reports a timeout during warm-up")
+
+    # ---- timed region: exactly K steps, per-step events on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(uuid) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
+        raise RuntimeError("device status word reports a timeout in the timed region")
+    total_ms = t_start.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if flush is not None:  # the flush writes sit between launches; count only kernel time
+        total_ms = sum(launch_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    ms_per_step = max_ms / args.steps
+    value = w.flops * args.steps * world / (max_ms * 1e-3) / 1e12
+    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 50))
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lseh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
+        oh.copy_(od, non_blocking=True)
+        lseh.copy_(lsed, non_blocking=True)
+
+    e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = w.flops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = q.numel() * q.element_size() + lseh.numel() * 4
+
+    if rank == 0:
+        peak, peak_sus, peak_src = measured_peak()
+        achieved = w.flops / (avg_launch_ms * 1e-3) / 1e12
+        traffic, traffic_how = recorded_traffic(w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": workload_config(w),
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
+                         "frac_of_sustained_peak": achieved / peak_sus,
+                         "algorithmic_bytes": w.min_hbm_bytes,
+                         "traffic_source": traffic_how},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "clocks": clocks.summary(),
+            "gpu_launches": args.steps,
+            "kernel_source_hash": kernel_source_hash(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            from tests.parity import metrics, passes
+
+            rows, o_ref, lse_ref, dt, threads = oracle_row_sample(w, q, k, v, args.cpu_seconds)
+            o_gpu = od.cpu().to(torch.float64).numpy()
+            l_gpu = lsed.cpu().to(torch.float64).numpy()
+            m = metrics(o_gpu[rows[:, 0], rows[:, 2], rows[:, 1]], l_gpu[rows[:, 0], rows[:, 1], rows[:, 2]],
+                        o_ref, lse_ref)
+            line["cpu_baseline"] = {
+                "value": row_flops(w, rows) / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "sample": f"{len(rows)} random (b,h,i) rows of the same inputs, fp64, {dt:.1f} s"}
+            line["parity"] = dict(m, rows=int(len(rows)), passes=passes(m))
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,145 @@
-"""B200-native exact attention forward (fused, online softmax, per-row LSE)."""
+"""B200-native exact attention forward: O = softmax(scale * Q K^T [+ causal]) V and per-row LSE.
+
+Thin Python binding over the C ABI in ``include/fa.h`` (library
+``libfa_b200.so``, built in-tree for sm_100a). This module only marshals
+arguments (pointers, sizes, the current CUDA stream); every step of the
+computation runs in the library's CUDA kernel. There is no fallback: if the
+library is missing or the device is not an sm_100 GPU, calls raise.
+
+Tensors use the [B, N, H, D] layout (contiguous, bf16 or fp16, D in {64, 128});
+LSE is float32 [B, H, N] in natural-log units of the scaled logits.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = ["fwd", "fwd_into", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
+           "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
+           "FA_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+
+FA_BF16 = 0
+FA_FP16 = 1
+
+# Every entry point declared in include/fa.h.
+EXPORTED_SYMBOLS = ("fa_status_string", "fa_fwd", "fa_status_sync", "fa_fwd_debug")
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
+_lib = None
+
+
+class FaError(RuntimeError):
+    """A non-OK status from the C library."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+
+
+def library_path() -> str:
+    return _LIB_FILE
+
+
+def load_library():
+    """Load the in-tree CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_FILE):
+        raise RuntimeError(f"CUDA library {_LIB_FILE} is missing; build it with "
+                           "`python -m exact_attention_151_b200.build`")
+    lib = ctypes.CDLL(_LIB_FILE)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.fa_status_string.argtypes = [i32]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    fwd_args = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, i32, i32, vp]
+    lib.fa_fwd.argtypes = fwd_args
+    lib.fa_fwd.restype = i32
+    lib.fa_fwd_debug.argtypes = fwd_args + [ctypes.c_uint64, i32]
+    lib.fa_fwd_debug.restype = i32
+    lib.fa_status_sync.argtypes = [vp]
+    lib.fa_status_sync.restype = i32
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().fa_status_string(int(code)).decode()
+
+
+def fwd_ptr(q: int, k: int, v: int, o: int, lse: int, B: int, N: int, H: int, D: int, scale: float,
+            causal: bool, dtype: int, stream: int, *, wait_limit_ns: int | None = None,
+            withhold_v_load: bool = False) -> int:
+    """Raw C-ABI call with integer device pointers; returns the fa_status code."""
+    lib = load_library()
+    if wait_limit_ns is None and not withhold_v_load:
+        return lib.fa_fwd(q, k, v, o, lse, B, N, H, D, ctypes.c_float(scale), int(bool(causal)), int(dtype),
+                          stream)
+    return lib.fa_fwd_debug(q, k, v, o, lse, B, N, H, D, ctypes.c_float(scale), int(bool(causal)), int(dtype),
+                            stream, int(wait_limit_ns or 0), int(bool(withhold_v_load)))
+
+
+def status_sync(stream: int | None = None) -> int:
+    """Synchronise the stream, then read and clear the device status word."""
+    import torch
+
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return load_library().fa_status_sync(s)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
+
+
+def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, **debug) -> None:
+    """Run the forward into caller-provided ``o`` ([B,N,H,D]) and ``lse`` (fp32 [B,H,N])."""
+    import torch
+
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
+        raise ValueError("q, k, v, o must share one [B, N, H, D] shape")
+    B, N, H, D = q.shape
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
+        raise TypeError("q, k, v and o must share one dtype")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, D,
+                     float(scale), causal, code, stream, **debug)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd")
+
+
+def fwd(q, k, v, scale: float | None = None, causal: bool = False):
+    """Exact attention forward. Returns (o [B,N,H,D] like q, lse float32 [B,H,N])."""
+    import torch
+
+    B, N, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fwd_into(q, k, v, o, lse, scale=scale, causal=causal)
+    return o, lse

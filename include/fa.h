@@ -1,0 +1,110 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) fused exact-attention forward.
+ *
+ * The operation (one call):
+ *   O[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) * v[b,j,h,:]
+ *   LSE[b,h,i] = ln sum_j exp(scale * q[b,i,h,:] . k[b,j,h,:])
+ * over the visible keys j (all j < N, or j <= i when causal).
+ *   - The formula and its four steps (similarity, scaling, softmax, weighted
+ *     sum of V): llmtrend.com, "FlashAttention ...", self-attention section.
+ *   - Computed tile by tile with a running max / running sum (online
+ *     softmax), Q/K/V loaded once and no N x N matrix written to memory:
+ *     jsqmd.com "Flash Attention applications", core-mechanism section
+ *     (kernel fusion, tiling + streaming); tuning handbook ch. 3,
+ *     "engineering implementation" section (tiled routine with lse).
+ *   - Causal masking skips future positions: handbook ch. 3, practical notes.
+ *   - The per-row log-sum-exp output (lse of shape [B, H, N]): the handbook's
+ *     tiled routine, which keeps and updates lse per query row.
+ *   - API shape (q, k, v, causal): mlqm.cn FA1/FA2 comparison, section 6.1.
+ *
+ * Layout (all buffers device memory, owned by the caller, never retained):
+ *   q, k, v, o : [B, N, H, D] contiguous, one 16-bit dtype (bf16 or fp16),
+ *                element (b,n,h,d) at ((b*N + n)*H + h)*D + d.
+ *   lse        : float32 [B, H, N] contiguous, natural log of the scaled logits.
+ *   Base pointers must be 16-byte aligned.
+ *
+ * The library makes no device allocation per call; its only device-side
+ * state is one status word per device (a static __device__ variable) that
+ * records asynchronous faults (see fa_status_sync).
+ *
+ * Errors: host-detectable errors return a status WITHOUT launching anything
+ * and leave o and lse untouched. A successful return means the work was
+ * enqueued on `stream`; device-side timeouts are reported later through
+ * fa_status_sync. No C++ exception ever crosses this boundary.
+ */
+#ifndef FA_B200_FA_H_
+#define FA_B200_FA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same ABI as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+  FA_BF16 = 0, /* bfloat16 inputs and output */
+  FA_FP16 = 1  /* IEEE binary16 inputs and output */
+} fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, unknown dtype, non-finite scale */
+  FA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, sizes beyond the limits below, or not an sm_100 device */
+  FA_ERR_MISALIGNED = 3,  /* a base pointer is not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime call failed (no device, launch failure, ...) */
+  FA_ERR_TIMEOUT = 5      /* a device-side wait ran out (reported by fa_status_sync) */
+} fa_status;
+
+/* Limits checked before launch: 1 <= D in {64,128}; B*H <= 2^31-1;
+ * N <= 2^31-1; each of q/k/v/o spans < 2^40 bytes. */
+
+/* Static, human-readable name of a status code; never NULL. */
+const char* fa_status_string(fa_status status);
+
+/*
+ * fa_fwd - fused exact-attention forward, enqueued on `stream`.
+ *
+ *   q, k, v : device pointers, [B, N, H, D], dtype `dtype`        (read only)
+ *   o       : device pointer,  [B, N, H, D], dtype `dtype`        (written)
+ *   lse     : device pointer,  float32 [B, H, N]                  (written)
+ *   B, N, H : batch, sequence length (queries = keys), heads; >= 0
+ *   D       : head dimension, 64 or 128
+ *   scale   : multiplies q.k before the softmax (1/sqrt(D) in the pages); finite
+ *   causal  : nonzero -> key j is visible to query i iff j <= i (square, top-left aligned)
+ *   stream  : CUDA stream the kernel is launched on
+ *
+ * B*N*H == 0 is a valid no-op (FA_OK, nothing launched, pointers unchecked).
+ * Results are bitwise deterministic for identical inputs on one device.
+ * Returns FA_OK after enqueueing, or an error code without launching.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
+                 int64_t H, int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * fa_status_sync - synchronise `stream`, then read and clear this device's
+ * status word. Returns FA_OK, FA_ERR_TIMEOUT if a kernel on this device gave
+ * up on a bounded wait since the last call (its outputs are then invalid),
+ * or FA_ERR_CUDA if the synchronisation itself failed.
+ */
+fa_status fa_status_sync(fa_stream_t stream);
+
+/*
+ * fa_fwd_debug - fa_fwd with two test hooks (same arguments first).
+ *   wait_limit_ns   : give-up time for every device-side wait (0 = default, about 1 s).
+ *   withhold_v_load : nonzero -> the loader of the first CTA never issues the
+ *                     V load of its first key tile, so that CTA's waits run
+ *                     out and report FA_ERR_TIMEOUT through fa_status_sync
+ *                     (the GPU stays usable). For tests of the timeout path.
+ */
+fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
+                       int64_t H, int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream,
+                       uint64_t wait_limit_ns, int withhold_v_load);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H_ */

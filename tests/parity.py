@@ -1,0 +1,54 @@
+"""Parity metrics between the CUDA path and the fp64 oracle (test infrastructure).
+
+Tolerances (16-bit inputs, fp32 accumulation on the GPU):
+  max |O_gpu - O_ref|              <= 1e-2
+  ||O_gpu - O_ref||_2 / ||O_ref||_2 <= 5e-3
+  max |LSE_gpu - LSE_ref|          <= 1e-3
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+TOL_MAX_ABS_O = 1e-2
+TOL_REL_L2_O = 5e-3
+TOL_MAX_ABS_LSE = 1e-3
+
+
+def metrics(o_gpu, lse_gpu, o_ref, lse_ref) -> dict:
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    diff = o_gpu - o_ref
+    ref_norm = float(np.linalg.norm(o_ref))
+    return {
+        "max_abs_o": float(np.abs(diff).max()) if diff.size else 0.0,
+        "rel_l2_o": float(np.linalg.norm(diff) / ref_norm) if ref_norm > 0 else float(np.linalg.norm(diff)),
+        "max_abs_lse": float(np.abs(lse_gpu - lse_ref).max()) if lse_ref.size else 0.0,
+        "finite": bool(np.isfinite(o_gpu).all() and np.isfinite(lse_gpu).all()),
+    }
+
+
+def passes(m: dict) -> bool:
+    return (m["finite"] and m["max_abs_o"] <= TOL_MAX_ABS_O and m["rel_l2_o"] <= TOL_REL_L2_O
+            and m["max_abs_lse"] <= TOL_MAX_ABS_LSE)
+
+
+def sample_rows(B: int, H: int, N: int, per_head_random: int, seed: int = 0, heads: list | None = None,
+                block: int = 128) -> np.ndarray:
+    """(b, h, i) triples covering, for each chosen head, the first and last rows,
+    the rows on both sides of every `block` boundary, and random rows."""
+    rng = np.random.default_rng(seed)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    edge = {0, 1, N - 2, N - 1}
+    for t in range(block, N, block):
+        edge.update((t - 1, t))
+    edge = sorted(i for i in edge if 0 <= i < N)
+    out = []
+    for b, h in heads:
+        rows = set(edge)
+        rows.update(rng.integers(0, N, size=per_head_random).tolist())
+        out.extend((b, h, i) for i in sorted(rows))
+    return np.array(out, dtype=np.int64)

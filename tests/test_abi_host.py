@@ -1,0 +1,59 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/fa.h declares, and rejects bad arguments before it
+touches a device (no launch, error code returned)."""
+
+import os
+import re
+
+import pytest
+
+import exact_attention_151_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load_library()
+    syms = declared_symbols()
+    assert syms == sorted(fa.EXPORTED_SYMBOLS)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_status_strings():
+    for code in range(6):
+        assert fa.status_string(code).startswith("FA_")
+    assert "UNKNOWN" in fa.status_string(99)
+
+
+# Argument combinations that must fail validation before any device call.
+P = 1 << 20  # a 16-byte aligned, never dereferenced address
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, P, P, P, P, 1, 16, 1, 64), fa.FA_ERR_INVALID_ARG),       # null q
+    ((P, P, P, P, 0, 1, 16, 1, 64), fa.FA_ERR_INVALID_ARG),       # null lse
+    ((P, P, P, P, P, -1, 16, 1, 64), fa.FA_ERR_INVALID_ARG),      # negative B
+    ((P, P, P, P, P, 1, -16, 1, 64), fa.FA_ERR_INVALID_ARG),      # negative N
+    ((P, P, P, P, P, 1, 16, 1, 96), fa.FA_ERR_UNSUPPORTED),       # D = 96
+    ((P, P, P, P, P, 1, 16, 1, 256), fa.FA_ERR_UNSUPPORTED),      # D = 256
+    ((P + 8, P, P, P, P, 1, 16, 1, 64), fa.FA_ERR_MISALIGNED),    # q not 16-byte aligned
+    ((P, P, P, P, P + 4, 1, 16, 1, 64), fa.FA_ERR_MISALIGNED),    # lse not 16-byte aligned
+    ((0, 0, 0, 0, 0, 0, 16, 1, 64), fa.FA_OK),                    # empty batch: no-op
+    ((0, 0, 0, 0, 0, 1, 0, 1, 64), fa.FA_OK),                     # empty sequence: no-op
+    ((0, 0, 0, 0, 0, 1, 16, 0, 64), fa.FA_OK),                    # no heads: no-op
+])
+def test_argument_validation(args, expect):
+    assert fa.fwd_ptr(*args, 0.125, False, fa.FA_BF16, 0) == expect
+
+
+def test_bad_dtype_and_scale():
+    assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, 0.125, False, 7, 0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, float("inf"), False, fa.FA_BF16, 0) == fa.FA_ERR_INVALID_ARG
+    assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, float("nan"), True, fa.FA_FP16, 0) == fa.FA_ERR_INVALID_ARG
