@@ -87,13 +87,22 @@ struct Cfg {
   static constexpr int kBarKVEmpty = kBarVFull + kStages;
   static constexpr int kBarSFull = kBarKVEmpty + kStages;  // [2]
   static constexpr int kBarPFull = kBarSFull + 2;          // [2]
-  static constexpr int kBarODone = kBarPFull + 2;
-  static constexpr int kBarDrain = kBarODone + 1;
+  static constexpr int kBarODone = kBarPFull + 2;   // one phase per PV but the last
+  static constexpr int kBarOFinal = kBarODone + 1;  // single phase: the last PV
+  static constexpr int kBarDrain = kBarOFinal + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024 B
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+
+// Tile (query tile qt, key tile j) whose P is applied as P16 + (P - P16).
+// Only the first key tile of the first query tile holds rows that see few
+// keys (causal rows 0..127, or every row when N <= 128); there a single
+// 16-bit rounding of P would weigh on the result about as much as the final
+// rounding of O, so the residual is added with a second MMA pass. Elsewhere
+// every row averages over more than 128 keys and the residual is negligible.
+__device__ __forceinline__ bool split_p_tile(int qt, int j) { return qt == 0 && j == 0; }
 
 struct WaitCtl {
   volatile int* abort;
@@ -172,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarPFull + i), 128);
     }
     mbar_init(bar(C::kBarODone), 1);
+    mbar_init(bar(C::kBarOFinal), 1);
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -264,7 +274,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = smem_desc_sw128(v_smem(sp) + kk * 2048, C::kSlabBytes, 1024);
             mma_ts(tmem + kOCol, p_tmem + kk * 8, bd, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(C::kBarODone));
+          if (split_p_tile(qt, jp)) {
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              const uint64_t bd = smem_desc_sw128(v_smem(sp) + kk * 2048, C::kSlabBytes, 1024);
+              mma_ts(tmem + kOCol, p_tmem + 64 + kk * 8, bd, idesc_pv, 1u);
+            }
+          }
+          // A parity wait is only unambiguous while the waiter is at most one
+          // phase behind, which holds for the rescale waits on o_done (tile j
+          // waits for PV_{j-1} after S_j, itself ordered after PV_{j-2}) but not
+          // for the epilogue; the last PV therefore signals its own barrier.
+          if (jp + 1 < n_kv) {
+            mma_commit(bar(C::kBarODone));
+          } else {
+            mma_commit(bar(C::kBarOFinal));
+          }
           if (jp + C::kStages < n_kv) mma_commit(bar(C::kBarKVEmpty + sp));
         }
       }
@@ -341,6 +366,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P_j (16-bit pairs, key 2i in the low half of column i) over S_j's first 64 columns.
       tmem_st32(tmem + lane_base + sbuf, pk[0]);
       tmem_st32(tmem + lane_base + sbuf + 32, pk[1]);
+      if (split_p_tile(qt, j)) {
+        // Rows with only a few keys: also store the rounding residual P - P16
+        // over the other 64 columns; the MMA adds it with a second pass.
+        uint32_t lo[2][32];
+#pragma unroll
+        for (int c = 0; c < kBN; c += 2) {
+          const float p0 = ex2_approx(x[c] - m_used);
+          const float p1 = ex2_approx(x[c + 1] - m_used);
+          const float2 hi = unpack2<FP16>(pk[(c / 2) / 32][(c / 2) % 32]);
+          lo[(c / 2) / 32][(c / 2) % 32] = pack2<FP16>(p0 - hi.x, p1 - hi.y);
+        }
+        tmem_st32(tmem + lane_base + sbuf + 64, lo[0]);
+        tmem_st32(tmem + lane_base + sbuf + 96, lo[1]);
+      }
       tmem_wait_st();
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
         // O holds the sum up to tile j-1 under the old max: wait for PV_{j-1}, then scale.
@@ -361,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + (j & 1)));
     }
-    if (ok) ok = warp_wait_bar(bar(C::kBarODone), static_cast<uint32_t>((n_kv - 1) & 1), wc);
+    if (ok) ok = warp_wait_bar(bar(C::kBarOFinal), 0, wc);
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_sum;

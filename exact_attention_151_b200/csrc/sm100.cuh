@@ -205,5 +205,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 
+// Inverse of pack2: the two 16-bit values of `v` widened to float (exact).
+template <bool FP16>
+__device__ __forceinline__ float2 unpack2(uint32_t v) {
+  float2 r;
+  if constexpr (FP16) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(v));
+  } else {
+    r.x = __uint_as_float(v << 16);
+    r.y = __uint_as_float(v & 0xffff0000u);
+  }
+  return r;
+}
+
 }  // namespace sm100
 }  // namespace fa
