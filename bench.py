@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
 DEFAULT_WORKLOAD = "llama7b_b4h32n2048d128_causal"
-KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_151_b200", "csrc", f) for f in ("fa_fwd.cu", "sm100.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_151_b200", "csrc", f) for f in ("fa_fwd.cu", "fa_fwd_kernel.cuh", "sm100.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_PEAK_TFLOPS = 1590.0
 

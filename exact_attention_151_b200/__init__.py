@@ -31,7 +31,7 @@ FA_BF16 = 0
 FA_FP16 = 1
 
 # Every entry point declared in include/fa.h.
-EXPORTED_SYMBOLS = ("fa_status_string", "fa_fwd", "fa_status_sync", "fa_fwd_debug")
+EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_status_sync", "fa_fwd_debug")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -43,7 +43,8 @@ class FaError(RuntimeError):
 
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        detail = last_error() if code == FA_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(code)} (code {code})" + (f" [{detail}]" if detail else ""))
 
 
 def library_path() -> str:
@@ -62,6 +63,8 @@ def load_library():
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.fa_status_string.argtypes = [i32]
     lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_error.argtypes = []
+    lib.fa_last_error.restype = ctypes.c_char_p
     fwd_args = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, i32, i32, vp]
     lib.fa_fwd.argtypes = fwd_args
     lib.fa_fwd.restype = i32
@@ -71,6 +74,11 @@ def load_library():
     lib.fa_status_sync.restype = i32
     _lib = lib
     return lib
+
+
+def last_error() -> str:
+    """Detail of the last FA_ERR_CUDA on this thread ("" if none)."""
+    return load_library().fa_last_error().decode()
 
 
 def status_string(code: int) -> str:

@@ -1,0 +1,538 @@
+// fa_fwd_kernel.cuh - the fused exact-attention forward kernel for sm_100a.
+//
+// What one CTA computes: O and LSE for a 256-row query block (two 128-row
+// query tiles Q0, Q1) of one (batch, head), streaming over the visible
+// 128-key tiles with an online softmax (running max and running sum per
+// query row), so no N x N score or probability matrix reaches global memory:
+//   * tiling Q / K / V and accumulating the softmax numerator and denominator
+//     block by block: llmtrend.com FlashAttention page, "how it works";
+//   * running max / running sum, rescaling the partial output: tuning handbook
+//     ch. 3, "core idea" and the tiled routine in "engineering implementation";
+//     jsqmd.com page, tiling + streaming;
+//   * one fused kernel for QK^T -> softmax -> PV: jsqmd.com page, kernel fusion;
+//   * K/V for the next tiles loaded while the current one is computed:
+//     mlqm.cn FA1/FA2 comparison, section 2.2;
+//   * work split over query blocks x batch x heads with K/V shared by the
+//     block's rows: mlqm.cn section 2.1 (FA2 partition);
+//   * causal attention skips future positions: handbook ch. 3, practical notes.
+//
+// Blackwell mapping (prior art on the pages targets Ampere; this is not it):
+//   warp 9 (loader)    TMA 4-D tiled loads: Q0 and Q1 once, K_j and V_j into
+//                      separate rings of 128B-swizzled shared-memory tiles;
+//   warp 8 (MMA)       one thread issues tcgen05.mma in the order
+//                        S0(j), PV1(j-1), S1(j), PV0(j)
+//                      so that while one softmax warpgroup works on its
+//                      scores the tensor cores serve the other query tile;
+//                      S_i = Q_i K_j^T lands in TMEM (fp32), O_i += P_i V_j
+//                      reads P_i from TMEM (16-bit) and V_j from shared memory;
+//   warps 0-3 / 4-7    softmax warpgroup i for query tile i: one query row per
+//                      thread (TMEM lane = row), so row max and row sum need
+//                      no shuffles; writes P_i over the first half of S_i's
+//                      columns; rescales O_i when its row max grew; finally
+//                      normalises O_i and writes O and LSE.
+// Because S_i(j) is issued after PV_i(j-1), the completion of S_i(j) implies
+// that PV_i(j-1) has finished, so the O_i rescale needs no extra barrier.
+//
+// Online-softmax bookkeeping (base 2, x = s * scale * log2(e)): m is only
+// raised when a tile's max exceeds it by more than kRescaleThreshold, so
+// P = 2^(x - m) stays below 2^threshold, which 16-bit P and fp32 sums hold
+// easily; O and l always share the same m, so O / l and
+// LSE = (m + log2 l) * ln 2 are exact up to rounding.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+using namespace sm100;
+
+// Device status word: bit 0 set when some wait ran out. Read and cleared by
+// fa_status_sync. A static __device__ variable, so the library allocates nothing.
+__device__ unsigned int g_status_word;
+
+constexpr int kTile = 128;        // query rows per tile = keys per tile = TMEM lanes
+constexpr int kBlockRows = 256;   // query rows per CTA (two tiles)
+constexpr int kThreads = 384;     // 12 warps = 3 warpgroups
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;      // warps 10 and 11 only keep warpgroup 2 whole
+// Registers per thread: the launch gives every thread kLaunchRegs (what ptxas
+// allots for 384 threads); warpgroup 2 (MMA, loader) then gives registers back
+// and the two softmax warpgroups take them. The shares must not exceed the
+// launch pool, or the increase would wait forever:
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kControlRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kMaxPolls = 1u << 28;
+constexpr uint64_t kDrainLimitNs = 20ull * 1000 * 1000;
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kHalves = D / 64;        // 64-element (128 B) column slabs per row
+  static constexpr int kSlabBytes = 128 * 128;  // one slab: 128 rows x 128 B
+  static constexpr int kTileBytes = kHalves * kSlabBytes;
+  static constexpr int kKStages = (D == 128) ? 2 : 4;
+  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kQOff = 0;  // Q0 then Q1
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKFull = kBarQ + 1;
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;  // [2]: S_i ready
+  static constexpr int kBarPFull = kBarSFull + 2;          // [2]: P_i written (128 arrivals)
+  static constexpr int kBarOFinal = kBarPFull + 2;         // [2]: last PV_i done (single phase)
+  static constexpr int kBarDrain = kBarOFinal + 2;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024 B
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // TMEM columns
+  __host__ __device__ static constexpr uint32_t col_s(int i) { return static_cast<uint32_t>(i) * 128u; }
+  __host__ __device__ static constexpr uint32_t col_o(int i) { return 256u + static_cast<uint32_t>(i * D); }
+  static_assert(256 + 2 * D <= kTmemCols, "TMEM budget");
+};
+
+struct WaitCtl {
+  volatile int* abort;
+  uint64_t limit_ns;
+};
+
+// Bounded wait for the phase of `bar` with `parity`. Returns false if this
+// CTA is aborting or the wait ran out (which starts the abort and records the
+// timeout in the status word).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, WaitCtl w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1; it < kMaxPolls; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort) return false;
+    if ((it & 15u) == 0 && globaltimer_ns() - t0 > w.limit_ns) break;
+  }
+  *w.abort = 1;
+  atomicOr(&g_status_word, 1u);
+  return false;
+}
+
+// Short bounded wait used while tearing down (loads and MMAs in flight).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; it < kMaxPolls; ++it) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((it & 15u) == 0 && globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+// Warp-uniform wrapper: every lane polls; the warp proceeds only if all did.
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, WaitCtl w) {
+  const bool ok = wait_bar(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Tile (query tile qt, key tile j) whose P is applied as P16 + (P - P16).
+// Only the first key tile of the first query tile holds rows that see few
+// keys (causal rows 0..127, or every row when N <= 128); there a single
+// 16-bit rounding of P would weigh on the result about as much as the final
+// rounding of O, so the residual is added with a second MMA pass. Elsewhere
+// every row averages over more than 128 keys and the residual is negligible.
+__device__ __forceinline__ bool split_p_tile(int qt, int j) { return qt == 0 && j == 0; }
+
+// Pairs of score columns whose exp2 runs on the FMA pipe instead of the
+// MUFU unit (every fourth pair), relieving the exp unit, which the tensor
+// cores otherwise outrun at D = 128.
+__device__ __forceinline__ constexpr bool emulated_pair(int pair) { return (pair & 3) == 3; }
+
+// One row of one score tile: p = 2^(s * c - m) for the 128 keys, stored to
+// TMEM at `s_col` as 16-bit pairs (key 2i in the low half of column i) over
+// 64 columns; with SPLIT also the rounding residual p - p16 over the next 64
+// columns. Returns the fp32 sum of p. Each score register dies as soon as its
+// pair is packed, which keeps the live set near one row of scores.
+template <bool FP16, bool SPLIT>
+__device__ __forceinline__ float softmax_exp_store(float (&s)[kTile], float c, float m, uint32_t s_col) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  uint32_t pk[2][32];
+  uint32_t lo[SPLIT ? 2 : 1][32];
+#pragma unroll
+  for (int pr = 0; pr < kTile / 2; ++pr) {
+    const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
+    float2 p;
+    if (emulated_pair(pr)) {
+      p = exp2_poly2(x);
+    } else {
+      p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    }
+    if (pr & 1) {
+      acc1 = fadd2(acc1, p);
+    } else {
+      acc0 = fadd2(acc0, p);
+    }
+    const uint32_t h = pack2<FP16>(p.x, p.y);
+    pk[pr / 32][pr % 32] = h;
+    if constexpr (SPLIT) {
+      const float2 hf = unpack2<FP16>(h);
+      lo[pr / 32][pr % 32] = pack2<FP16>(p.x - hf.x, p.y - hf.y);
+    }
+  }
+  tmem_st32(s_col, pk[0]);
+  tmem_st32(s_col + 32, pk[1]);
+  if constexpr (SPLIT) {
+    tmem_st32(s_col + 64, lo[0]);
+    tmem_st32(s_col + 96, lo[SPLIT ? 1 : 0]);
+  }
+  const float2 acc = fadd2(acc0, acc1);
+  return acc.x + acc.y;
+}
+
+// Problem description passed by value.
+struct Params {
+  uint16_t* out;
+  float* lse;
+  int N, H;
+  int n_tiles;   // ceil(N / 128)
+  int n_blocks;  // ceil(N / 256)
+  float scale_log2;
+  int causal;
+  unsigned long long wait_limit_ns;
+  int withhold_v_load;
+};
+
+template <int D, bool FP16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const Params prm) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto q_smem = [&](int i) { return sbase + C::kQOff + i * C::kTileBytes; };
+  auto k_smem = [&](int s) { return sbase + C::kKOff + s * C::kTileBytes; };
+  auto v_smem = [&](int s) { return sbase + C::kVOff + s * C::kTileBytes; };
+  auto bar = [&](int i) { return sbase + C::kBarOff + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int N = prm.N;
+  const int causal = prm.causal;
+
+  // Work item: CTAs of one (b, h) are adjacent (K/V reuse in L2); for causal
+  // attention the heaviest query blocks of each head go first.
+  const int bh = blockIdx.x / prm.n_blocks;
+  const int t = blockIdx.x % prm.n_blocks;
+  const int mb = causal ? (prm.n_blocks - 1 - t) : t;
+  const int b = bh / prm.H;
+  const int h = bh % prm.H;
+  const int qt0 = 2 * mb;
+  const int qt1 = 2 * mb + 1;
+  const bool q1_valid = qt1 < prm.n_tiles;
+  // key tiles visited, and the last key tile of each query tile
+  const int last0 = causal ? qt0 : prm.n_tiles - 1;
+  const int last1 = q1_valid ? (causal ? qt1 : prm.n_tiles - 1) : -1;
+  const int n_kv = (last1 > last0 ? last1 : last0) + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::kBarQ), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::kBarSFull + i), 1);
+      mbar_init(bar(C::kBarPFull + i), 128);
+      mbar_init(bar(C::kBarOFinal + i), 1);
+    }
+    mbar_init(bar(C::kBarDrain), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, prm.wait_limit_ns};
+
+  if (warp >= 8) {
+    regs_decrease<kControlRegs>();
+    if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
+      for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, (qt0 + i) * kTile, b, bar(C::kBarQ));
+      const bool withhold = prm.withhold_v_load && blockIdx.x == 0;
+      int nk = 0, nv = 0;  // K and V tiles issued
+      for (int j = 0; j < n_kv; ++j) {
+        const int sk = j % C::kKStages;
+        if (j >= C::kKStages &&
+            !wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((j / C::kKStages) & 1) ^ 1), wc))
+          break;
+        mbar_arrive_expect_tx(bar(C::kBarKFull + sk), C::kTileBytes);
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, j * kTile, b, bar(C::kBarKFull + sk));
+        nk = j + 1;
+        const int sv = j % C::kVStages;
+        if (j >= C::kVStages &&
+            !wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((j / C::kVStages) & 1) ^ 1), wc))
+          break;
+        if (!(withhold && j == 0)) {
+          mbar_arrive_expect_tx(bar(C::kBarVFull + sv), C::kTileBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_4d(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, j * kTile, b, bar(C::kBarVFull + sv));
+        }
+        nv = j + 1;
+      }
+      // Let every load this thread issued land before shared memory is
+      // released (immediate in a normal run, where all were consumed): for
+      // each stage, wait for the phase of its last arming.
+      drain_wait(bar(C::kBarQ), 0);
+      for (int s = 0; s < C::kKStages && s < nk; ++s) {
+        const int jl = s + ((nk - 1 - s) / C::kKStages) * C::kKStages;
+        drain_wait(bar(C::kBarKFull + s), static_cast<uint32_t>((jl / C::kKStages) & 1));
+      }
+      for (int s = 0; s < C::kVStages && s < nv; ++s) {
+        const int jl = s + ((nv - 1 - s) / C::kVStages) * C::kVStages;
+        if (!(withhold && jl == 0)) drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((jl / C::kVStages) & 1));
+      }
+    }
+    __syncwarp();
+    } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = instr_desc_f16(kTile, kTile, FP16, false);
+      constexpr uint32_t idesc_pv = instr_desc_f16(kTile, D, FP16, true);
+      // S_i(j) = Q_i K_j^T  (K-major A and B, K = D in steps of 16)
+      auto issue_s = [&](int i, int sk) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kSlabBytes + (kk % 4) * 32;
+          mma_ss(tmem + C::col_s(i), smem_desc_sw128(q_smem(i) + off, 16, 1024),
+                 smem_desc_sw128(k_smem(sk) + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::kBarSFull + i));
+      };
+      // O_i += P_i(j) V_j  (P from TMEM, V MN-major, K = 128 keys in steps of 16)
+      auto issue_pv = [&](int i, int j, int sv, bool split) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
+                 smem_desc_sw128(v_smem(sv) + kk * 2048, C::kSlabBytes, 1024), idesc_pv,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        if (split) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + 64 + kk * 8,
+                   smem_desc_sw128(v_smem(sv) + kk * 2048, C::kSlabBytes, 1024), idesc_pv, 1u);
+        }
+      };
+      bool ok = wait_bar(bar(C::kBarQ), 0, wc);
+      for (int j = 0; ok && j <= n_kv; ++j) {
+        const int sk = j % C::kKStages;
+        if (j < n_kv) {
+          ok = wait_bar(bar(C::kBarKFull + sk), static_cast<uint32_t>((j / C::kKStages) & 1), wc);
+          if (!ok) break;
+          tc_fence_after();
+          if (j <= last0) issue_s(0, sk);
+        }
+        if (j >= 1 && j - 1 <= last1) {
+          // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
+          const int jp = j - 1, sv = jp % C::kVStages;
+          ok = wait_bar(bar(C::kBarPFull + 1), static_cast<uint32_t>(jp & 1), wc) &&
+               wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((jp / C::kVStages) & 1), wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, jp, sv, split_p_tile(qt1, jp));
+          if (jp == last1) mma_commit(bar(C::kBarOFinal + 1));
+          if (jp + C::kVStages < n_kv) mma_commit(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
+        }
+        if (j < n_kv) {
+          if (j <= last1) issue_s(1, sk);
+          if (j + C::kKStages < n_kv) mma_commit(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
+          if (j <= last0) {
+            const int sv = j % C::kVStages;
+            ok = wait_bar(bar(C::kBarPFull + 0), static_cast<uint32_t>(j & 1), wc) &&
+                 wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, j, sv, split_p_tile(qt0, j));
+            if (j == last0) mma_commit(bar(C::kBarOFinal + 0));
+            if (j > last1 && j + C::kVStages < n_kv) mma_commit(bar(C::kBarVEmpty + sv));
+          }
+        }
+      }
+      if (!ok) {
+        mma_commit(bar(C::kBarDrain));
+        drain_wait(bar(C::kBarDrain), 0);
+      }
+    }
+    __syncwarp();
+    }
+  } else {
+    regs_increase<kSoftmaxRegs>();
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp / 4;              // query tile of this warpgroup
+    const int qt = qt0 + wg;
+    const int last = wg == 0 ? last0 : last1;
+    const int quarter = warp % 4;         // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const int qi = qt * kTile + row;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + C::col_s(wg);
+    const uint32_t o_col = tmem + lane_base + C::col_o(wg);
+    const float c = prm.scale_log2;
+    const bool c_pos = c > 0.f;  // host guarantees c != 0
+    const float fill = c_pos ? -INFINITY : INFINITY;  // masked score: weight 2^-inf = 0
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j <= last; ++j) {
+      ok = warp_wait_bar(bar(C::kBarSFull + wg), static_cast<uint32_t>(j & 1), wc);
+      if (!ok) break;
+      tc_fence_after();
+      float s[kTile];
+      {
+        uint32_t r[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(s_col + q * 32, r[q]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < kTile; ++k) s[k] = __uint_as_float(r[k / 32][k % 32]);
+      }
+      const int kbase = j * kTile;
+      if ((causal && j == qt) || kbase + kTile > N) {
+        const int lastcol = (causal ? min(N - 1, qi) : (N - 1)) - kbase;  // last visible column
+#pragma unroll
+        for (int k = 0; k < kTile; ++k) s[k] = (k <= lastcol) ? s[k] : fill;
+      }
+      // tile max of x = s * c: c * max(s) for c > 0, c * min(s) for c < 0 (exact under rounding)
+      float e0, e1, e2, e3;
+      if (c_pos) {
+        e0 = max3f(s[0], s[1], s[2]);
+        e1 = max3f(s[3], s[4], s[5]);
+        e2 = max3f(s[6], s[7], s[8]);
+        e3 = max3f(s[9], s[10], s[11]);
+#pragma unroll
+        for (int k = 12; k < kTile - 8; k += 8) {
+          e0 = max3f(e0, s[k], s[k + 1]);
+          e1 = max3f(e1, s[k + 2], s[k + 3]);
+          e2 = max3f(e2, s[k + 4], s[k + 5]);
+          e3 = max3f(e3, s[k + 6], s[k + 7]);
+        }
+        e0 = max3f(e0, s[kTile - 4], s[kTile - 3]);
+        e1 = max3f(e1, s[kTile - 2], s[kTile - 1]);
+        e0 = max3f(e0, e1, fmaxf(e2, e3));
+      } else {
+        e0 = min3f(s[0], s[1], s[2]);
+        e1 = min3f(s[3], s[4], s[5]);
+        e2 = min3f(s[6], s[7], s[8]);
+        e3 = min3f(s[9], s[10], s[11]);
+#pragma unroll
+        for (int k = 12; k < kTile - 8; k += 8) {
+          e0 = min3f(e0, s[k], s[k + 1]);
+          e1 = min3f(e1, s[k + 2], s[k + 3]);
+          e2 = min3f(e2, s[k + 4], s[k + 5]);
+          e3 = min3f(e3, s[k + 6], s[k + 7]);
+        }
+        e0 = min3f(e0, s[kTile - 4], s[kTile - 3]);
+        e1 = min3f(e1, s[kTile - 2], s[kTile - 1]);
+        e0 = min3f(e0, e1, fminf(e2, e3));
+      }
+      const float m_tile = e0 * c;
+      const float m_new = fmaxf(m_used, m_tile);
+      const bool rescale = m_new > m_used + kRescaleThreshold;  // always true on the first tile
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx(m_used - m_new);  // 0 on the first tile (m_used = -inf)
+        l_sum *= alpha;
+        m_used = m_new;
+      }
+      // P = 2^(s * c - m) over the first 64 columns of S_i (16-bit pairs);
+      // the tile with few-key rows also gets its rounding residual.
+      if (split_p_tile(qt, j)) {
+        l_sum += softmax_exp_store<FP16, true>(s, c, m_used, s_col);
+      } else {
+        l_sum += softmax_exp_store<FP16, false>(s, c, m_used, s_col);
+      }
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        // O_i holds the sum up to tile j-1 under the old max; PV_i(j-1) has
+        // completed because S_i(j) was issued after it and has completed.
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(o_col + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 v = fmul2(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])),
+                                   make_float2(alpha, alpha));
+            o[k] = __float_as_uint(v.x);
+            o[k + 1] = __float_as_uint(v.y);
+          }
+          tmem_st32(o_col + q * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + wg));
+    }
+    if (last >= 0 && ok) ok = warp_wait_bar(bar(C::kBarOFinal + wg), 0, wc);
+    if (last >= 0 && ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_sum;
+      const bool row_valid = qi < N;
+      uint16_t* orow = prm.out + ((static_cast<int64_t>(b) * N + qi) * prm.H + h) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        tmem_ld32(o_col + q * 32, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 v = fmul2(make_float2(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1])),
+                                 make_float2(inv_l, inv_l));
+          pk[k] = pack2<FP16>(v.x, v.y);
+        }
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+      if (row_valid) prm.lse[(static_cast<int64_t>(b) * prm.H + h) * N + qi] = (m_used + lg2_approx(l_sum)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace fa

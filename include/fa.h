@@ -64,6 +64,11 @@ typedef enum {
 /* Static, human-readable name of a status code; never NULL. */
 const char* fa_status_string(fa_status status);
 
+/* Detail of the last FA_ERR_CUDA returned on the calling thread (the failing
+ * call and CUDA's message), or "" if none; owned by the library, valid until
+ * the thread's next call into it. */
+const char* fa_last_error(void);
+
 /*
  * fa_fwd - fused exact-attention forward, enqueued on `stream`.
  *
