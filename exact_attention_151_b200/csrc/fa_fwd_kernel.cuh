@@ -63,8 +63,8 @@ constexpr int kLoadWarp = 9;      // warps 10 and 11 only keep warpgroup 2 whole
 // and the two softmax warpgroups take them. The shares must not exceed the
 // launch pool, or the increase would wait forever:
 constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 224;
-constexpr uint32_t kControlRegs = 56;
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kControlRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.693147180559945309f;
@@ -276,33 +276,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kControlRegs>();
     if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loader
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
+    // The whole warp runs this loop (converged); one elected lane issues each
+    // barrier arm and TMA copy.
+    {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
+      __syncwarp();
+      mbar_arrive_expect_tx_elect(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
       for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, (qt0 + i) * kTile, b, bar(C::kBarQ));
+          tma_load_4d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, (qt0 + i) * kTile, b, bar(C::kBarQ));
       const bool withhold = prm.withhold_v_load && blockIdx.x == 0;
       int nk = 0, nv = 0;  // K and V tiles issued
       for (int j = 0; j < n_kv; ++j) {
         const int sk = j % C::kKStages;
         if (j >= C::kKStages &&
-            !wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((j / C::kKStages) & 1) ^ 1), wc))
+            !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((j / C::kKStages) & 1) ^ 1), wc))
           break;
-        mbar_arrive_expect_tx(bar(C::kBarKFull + sk), C::kTileBytes);
+        mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, j * kTile, b, bar(C::kBarKFull + sk));
+          tma_load_4d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, j * kTile, b, bar(C::kBarKFull + sk));
         nk = j + 1;
         const int sv = j % C::kVStages;
         if (j >= C::kVStages &&
-            !wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((j / C::kVStages) & 1) ^ 1), wc))
+            !warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((j / C::kVStages) & 1) ^ 1), wc))
           break;
         if (!(withhold && j == 0)) {
-          mbar_arrive_expect_tx(bar(C::kBarVFull + sv), C::kTileBytes);
+          mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
           for (int hf = 0; hf < C::kHalves; ++hf)
-            tma_load_4d(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, j * kTile, b, bar(C::kBarVFull + sv));
+            tma_load_4d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, j * kTile, b, bar(C::kBarVFull + sv));
         }
         nv = j + 1;
       }
@@ -322,38 +327,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop (converged, descriptors in uniform
+    // registers); one elected lane issues each tcgen05.mma and commit.
+    {
       constexpr uint32_t idesc_qk = instr_desc_f16(kTile, kTile, FP16, false);
       constexpr uint32_t idesc_pv = instr_desc_f16(kTile, D, FP16, true);
+      // Shared-memory descriptors are built once; a tile, stage or K step is
+      // reached by adding its byte offset / 16 to the start-address field
+      // (bits 0-13; shared addresses stay below 2^18, so nothing carries out).
+      // Keeping per-MMA work to one add lets issue keep up with the tensor pipe.
+      const uint64_t q_desc0 = smem_desc_sw128(q_smem(0), 16, 1024);
+      const uint64_t k_desc0 = smem_desc_sw128(k_smem(0), 16, 1024);
+      const uint64_t v_desc0 = smem_desc_sw128(v_smem(0), C::kSlabBytes, 1024);
+      constexpr uint64_t kTileStep = C::kTileBytes >> 4;
       // S_i(j) = Q_i K_j^T  (K-major A and B, K = D in steps of 16)
       auto issue_s = [&](int i, int sk) {
+        const uint64_t qa = q_desc0 + static_cast<uint64_t>(i) * kTileStep;
+        const uint64_t kb = k_desc0 + static_cast<uint64_t>(sk) * kTileStep;
+        const uint32_t d_tmem = tmem + C::col_s(i);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kSlabBytes + (kk % 4) * 32;
-          mma_ss(tmem + C::col_s(i), smem_desc_sw128(q_smem(i) + off, 16, 1024),
-                 smem_desc_sw128(k_smem(sk) + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
+          mma_ss_elect(d_tmem, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(C::kBarSFull + i));
+        mma_commit_elect(bar(C::kBarSFull + i));
       };
       // O_i += P_i(j) V_j  (P from TMEM, V MN-major, K = 128 keys in steps of 16)
       auto issue_pv = [&](int i, int j, int sv, bool split) {
+        const uint64_t vb = v_desc0 + static_cast<uint64_t>(sv) * kTileStep;
+        const uint32_t o_tmem = tmem + C::col_o(i);
+        const uint32_t p_tmem = tmem + C::col_s(i);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
-                 smem_desc_sw128(v_smem(sv) + kk * 2048, C::kSlabBytes, 1024), idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(o_tmem, p_tmem + kk * 8, vb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
         if (split) {
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + 64 + kk * 8,
-                   smem_desc_sw128(v_smem(sv) + kk * 2048, C::kSlabBytes, 1024), idesc_pv, 1u);
+            mma_ts_elect(o_tmem, p_tmem + 64 + kk * 8, vb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_pv, 1u);
         }
       };
-      bool ok = wait_bar(bar(C::kBarQ), 0, wc);
+      bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
       for (int j = 0; ok && j <= n_kv; ++j) {
         const int sk = j % C::kKStages;
         if (j < n_kv) {
-          ok = wait_bar(bar(C::kBarKFull + sk), static_cast<uint32_t>((j / C::kKStages) & 1), wc);
+          ok = warp_wait_bar(bar(C::kBarKFull + sk), static_cast<uint32_t>((j / C::kKStages) & 1), wc);
           if (!ok) break;
           tc_fence_after();
           if (j <= last0) issue_s(0, sk);
@@ -361,31 +379,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1 && j - 1 <= last1) {
           // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
           const int jp = j - 1, sv = jp % C::kVStages;
-          ok = wait_bar(bar(C::kBarPFull + 1), static_cast<uint32_t>(jp & 1), wc) &&
-               wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((jp / C::kVStages) & 1), wc);
+          ok = warp_wait_bar(bar(C::kBarPFull + 1), static_cast<uint32_t>(jp & 1), wc) &&
+               warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((jp / C::kVStages) & 1), wc);
           if (!ok) break;
           tc_fence_after();
           issue_pv(1, jp, sv, split_p_tile(qt1, jp));
-          if (jp == last1) mma_commit(bar(C::kBarOFinal + 1));
-          if (jp + C::kVStages < n_kv) mma_commit(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
+          if (jp == last1) mma_commit_elect(bar(C::kBarOFinal + 1));
+          if (jp + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
         }
         if (j < n_kv) {
           if (j <= last1) issue_s(1, sk);
-          if (j + C::kKStages < n_kv) mma_commit(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
+          if (j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
           if (j <= last0) {
             const int sv = j % C::kVStages;
-            ok = wait_bar(bar(C::kBarPFull + 0), static_cast<uint32_t>(j & 1), wc) &&
-                 wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc);
+            ok = warp_wait_bar(bar(C::kBarPFull + 0), static_cast<uint32_t>(j & 1), wc) &&
+                 warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc);
             if (!ok) break;
             tc_fence_after();
             issue_pv(0, j, sv, split_p_tile(qt0, j));
-            if (j == last0) mma_commit(bar(C::kBarOFinal + 0));
-            if (j > last1 && j + C::kVStages < n_kv) mma_commit(bar(C::kBarVEmpty + sv));
+            if (j == last0) mma_commit_elect(bar(C::kBarOFinal + 0));
+            if (j > last1 && j + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));
           }
         }
       }
       if (!ok) {
-        mma_commit(bar(C::kBarDrain));
+        mma_commit_elect(bar(C::kBarDrain));
         drain_wait(bar(C::kBarDrain), 0);
       }
     }
