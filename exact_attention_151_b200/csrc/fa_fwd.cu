@@ -147,6 +147,7 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.lse = lse;
   prm.N = static_cast<int>(N);
   prm.H = static_cast<int>(H);
+  prm.BH = static_cast<int>(B * H);
   prm.n_tiles = static_cast<int>((N + kTile - 1) / kTile);
   prm.n_blocks = static_cast<int>((N + kBlockRows - 1) / kBlockRows);
   // Softmax runs in base 2: x = s * scale * log2(e). A zero (or subnormal)

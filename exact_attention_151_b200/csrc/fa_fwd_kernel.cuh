@@ -55,6 +55,7 @@ __device__ unsigned int g_status_word;
 
 constexpr int kTile = 128;        // query rows per tile = keys per tile = TMEM lanes
 constexpr int kBlockRows = 256;   // query rows per CTA (two tiles)
+constexpr int kHeadGroup = 16;    // heads whose query blocks are interleaved in the grid order
 constexpr int kThreads = 384;     // 12 warps = 3 warpgroups
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;      // warps 10 and 11 only keep warpgroup 2 whole
@@ -90,8 +91,8 @@ struct Cfg {
   static constexpr int kBarVFull = kBarKEmpty + kKStages;
   static constexpr int kBarVEmpty = kBarVFull + kVStages;
   static constexpr int kBarSFull = kBarVEmpty + kVStages;  // [2]: S_i ready
-  static constexpr int kBarPFull = kBarSFull + 2;          // [2]: P_i written (128 arrivals)
-  static constexpr int kBarOFinal = kBarPFull + 2;         // [2]: last PV_i done (single phase)
+  static constexpr int kBarPFull = kBarSFull + 2;          // [2][2]: half h of P_i written (128 arrivals)
+  static constexpr int kBarOFinal = kBarPFull + 4;         // [2]: last PV_i done (single phase)
   static constexpr int kBarDrain = kBarOFinal + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag
@@ -148,51 +149,89 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Wai
 __device__ __forceinline__ bool split_p_tile(int qt, int j) { return qt == 0 && j == 0; }
 
 // Pairs of score columns whose exp2 runs on the FMA pipe instead of the
-// MUFU unit (every fourth pair), relieving the exp unit, which the tensor
-// cores otherwise outrun at D = 128.
+// MUFU unit (every fourth pair): the two softmax warpgroups share each SM
+// sub-partition's exp unit, which the tensor cores otherwise outrun.
 __device__ __forceinline__ constexpr bool emulated_pair(int pair) { return (pair & 3) == 3; }
 
-// One row of one score tile: p = 2^(s * c - m) for the 128 keys, stored to
-// TMEM at `s_col` as 16-bit pairs (key 2i in the low half of column i) over
-// 64 columns; with SPLIT also the rounding residual p - p16 over the next 64
-// columns. Returns the fp32 sum of p. Each score register dies as soon as its
-// pair is packed, which keeps the live set near one row of scores.
-template <bool FP16, bool SPLIT>
-__device__ __forceinline__ float softmax_exp_store(float (&s)[kTile], float c, float m, uint32_t s_col) {
+// Max (MAX) or min of one row of 128 scores: three-input max in four
+// independent chains.
+template <bool MAX>
+__device__ __forceinline__ float row_reduce(const float (&s)[kTile]) {
+  auto r3 = [](float a, float b, float c) { return MAX ? max3f(a, b, c) : min3f(a, b, c); };
+  float e0 = r3(s[0], s[1], s[2]);
+  float e1 = r3(s[3], s[4], s[5]);
+  float e2 = r3(s[6], s[7], s[8]);
+  float e3 = r3(s[9], s[10], s[11]);
+#pragma unroll
+  for (int k = 12; k < kTile - 8; k += 8) {
+    e0 = r3(e0, s[k], s[k + 1]);
+    e1 = r3(e1, s[k + 2], s[k + 3]);
+    e2 = r3(e2, s[k + 4], s[k + 5]);
+    e3 = r3(e3, s[k + 6], s[k + 7]);
+  }
+  e0 = r3(e0, s[kTile - 4], s[kTile - 3]);
+  e1 = r3(e1, s[kTile - 2], s[kTile - 1]);
+  return r3(e0, e1, MAX ? fmaxf(e2, e3) : fminf(e2, e3));
+}
+
+// Half h of one row of one score tile (keys 64h .. 64h+63): p = 2^(s * c - m),
+// packed to 16-bit pairs (key 2i in the low half of column i) and stored to
+// TMEM columns 32h .. 32h+31 of S_i in two 16-column chunks; with SPLIT also
+// the rounding residual p - p16 to columns 64 + 32h .. Returns the fp32 sum
+// of p. Each score register dies once its pair is packed.
+template <bool FP16, bool SPLIT, int HALF>
+__device__ __forceinline__ float softmax_exp_half(const float (&s)[kTile], float c, float m, uint32_t s_col) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m, -m);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-  uint32_t pk[2][32];
-  uint32_t lo[SPLIT ? 2 : 1][32];
 #pragma unroll
-  for (int pr = 0; pr < kTile / 2; ++pr) {
-    const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
-    float2 p;
-    if (emulated_pair(pr)) {
-      p = exp2_poly2(x);
-    } else {
-      p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+  for (int chunk = 0; chunk < 2; ++chunk) {
+    uint32_t pk[16];
+    uint32_t lo[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int pr = HALF * 32 + chunk * 16 + q;  // pair index in the row
+      const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
+      float2 p;
+      if (emulated_pair(pr)) {
+        p = exp2_poly2(x);
+      } else {
+        p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      if (q & 1) {
+        acc1 = fadd2(acc1, p);
+      } else {
+        acc0 = fadd2(acc0, p);
+      }
+      pk[q] = pack2<FP16>(p.x, p.y);
+      if constexpr (SPLIT) {
+        const float2 hf = unpack2<FP16>(pk[q]);
+        lo[q] = pack2<FP16>(p.x - hf.x, p.y - hf.y);
+      }
     }
-    if (pr & 1) {
-      acc1 = fadd2(acc1, p);
-    } else {
-      acc0 = fadd2(acc0, p);
-    }
-    const uint32_t h = pack2<FP16>(p.x, p.y);
-    pk[pr / 32][pr % 32] = h;
-    if constexpr (SPLIT) {
-      const float2 hf = unpack2<FP16>(h);
-      lo[pr / 32][pr % 32] = pack2<FP16>(p.x - hf.x, p.y - hf.y);
-    }
-  }
-  tmem_st32(s_col, pk[0]);
-  tmem_st32(s_col + 32, pk[1]);
-  if constexpr (SPLIT) {
-    tmem_st32(s_col + 64, lo[0]);
-    tmem_st32(s_col + 96, lo[SPLIT ? 1 : 0]);
+    tmem_st16(s_col + HALF * 32 + chunk * 16, pk);
+    if constexpr (SPLIT) tmem_st16(s_col + 64 + HALF * 32 + chunk * 16, lo);
   }
   const float2 acc = fadd2(acc0, acc1);
   return acc.x + acc.y;
+}
+
+// O row *= alpha in TMEM (warp-collective; D columns from o_col).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t o_col, float alpha) {
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) {
+    uint32_t o[32];
+    tmem_ld32(o_col + q * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+      const float2 v = fmul2(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), make_float2(alpha, alpha));
+      o[k] = __float_as_uint(v.x);
+      o[k + 1] = __float_as_uint(v.y);
+    }
+    tmem_st32(o_col + q * 32, o);
+  }
 }
 
 // Problem description passed by value.
@@ -200,6 +239,7 @@ struct Params {
   uint16_t* out;
   float* lse;
   int N, H;
+  int BH;        // B * H
   int n_tiles;   // ceil(N / 128)
   int n_blocks;  // ceil(N / 256)
   float scale_log2;
@@ -228,11 +268,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int N = prm.N;
   const int causal = prm.causal;
 
-  // Work item: CTAs of one (b, h) are adjacent (K/V reuse in L2); for causal
-  // attention the heaviest query blocks of each head go first.
-  const int bh = blockIdx.x / prm.n_blocks;
-  const int t = blockIdx.x % prm.n_blocks;
-  const int mb = causal ? (prm.n_blocks - 1 - t) : t;
+  int bh, level;
+  {
+    // Causal: heads in groups of kHeadGroup; inside a group, query-block level
+    // by level across the group's heads, heaviest first. The group's K/V stay
+    // in L2 while its CTAs run, and the last CTAs to start are the lightest.
+    const int per_group = kHeadGroup * prm.n_blocks;
+    const int full_groups = prm.BH / kHeadGroup;
+    const int x = static_cast<int>(blockIdx.x);
+    int g, hg, within;
+    if (x < full_groups * per_group) {
+      g = x / per_group;
+      hg = kHeadGroup;
+      within = x % per_group;
+    } else {
+      g = full_groups;
+      hg = prm.BH - full_groups * kHeadGroup;
+      within = x - full_groups * per_group;
+    }
+    level = within / hg;
+    bh = g * kHeadGroup + within % hg;
+  }
+  if (!causal) {
+    // equal work per block: keep all blocks of a head adjacent (K/V shared in L2)
+    bh = static_cast<int>(blockIdx.x) / prm.n_blocks;
+    level = static_cast<int>(blockIdx.x) % prm.n_blocks;
+  }
+  const int mb = causal ? (prm.n_blocks - 1 - level) : level;
   const int b = bh / prm.H;
   const int h = bh % prm.H;
   const int qt0 = 2 * mb;
@@ -255,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::kBarSFull + i), 1);
-      mbar_init(bar(C::kBarPFull + i), 128);
+      mbar_init(bar(C::kBarPFull + 2 * i), 128);
+      mbar_init(bar(C::kBarPFull + 2 * i + 1), 128);
       mbar_init(bar(C::kBarOFinal + i), 1);
     }
     mbar_init(bar(C::kBarDrain), 1);
@@ -352,20 +415,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit_elect(bar(C::kBarSFull + i));
       };
-      // O_i += P_i(j) V_j  (P from TMEM, V MN-major, K = 128 keys in steps of 16)
-      auto issue_pv = [&](int i, int j, int sv, bool split) {
+      // O_i += P_i(j) V_j for keys 64h .. 64h+63 (P from TMEM, V MN-major,
+      // K in steps of 16); the split tile adds the residual pass.
+      auto issue_pv_half = [&](int i, int j, int sv, bool split, int h) {
         const uint64_t vb = v_desc0 + static_cast<uint64_t>(sv) * kTileStep;
         const uint32_t o_tmem = tmem + C::col_o(i);
         const uint32_t p_tmem = tmem + C::col_s(i);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
+        for (int q = 0; q < 4; ++q) {
+          const int kk = 4 * h + q;
           mma_ts_elect(o_tmem, p_tmem + kk * 8, vb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_pv,
                        (j > 0 || kk > 0) ? 1u : 0u);
+        }
         if (split) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
+          for (int q = 0; q < 4; ++q) {
+            const int kk = 4 * h + q;
             mma_ts_elect(o_tmem, p_tmem + 64 + kk * 8, vb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_pv, 1u);
+          }
         }
+      };
+      // Both halves of PV_i(j): each waits for its half of P.
+      auto issue_pv = [&](int i, int j, int sv, bool split) -> bool {
+        if (!warp_wait_bar(bar(C::kBarPFull + 2 * i), static_cast<uint32_t>(j & 1), wc) ||
+            !warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc))
+          return false;
+        tc_fence_after();
+        issue_pv_half(i, j, sv, split, 0);
+        if (!warp_wait_bar(bar(C::kBarPFull + 2 * i + 1), static_cast<uint32_t>(j & 1), wc)) return false;
+        tc_fence_after();
+        issue_pv_half(i, j, sv, split, 1);
+        return true;
       };
       bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
       for (int j = 0; ok && j <= n_kv; ++j) {
@@ -379,11 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1 && j - 1 <= last1) {
           // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
           const int jp = j - 1, sv = jp % C::kVStages;
-          ok = warp_wait_bar(bar(C::kBarPFull + 1), static_cast<uint32_t>(jp & 1), wc) &&
-               warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((jp / C::kVStages) & 1), wc);
+          ok = issue_pv(1, jp, sv, split_p_tile(qt1, jp));
           if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, jp, sv, split_p_tile(qt1, jp));
           if (jp == last1) mma_commit_elect(bar(C::kBarOFinal + 1));
           if (jp + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
         }
@@ -392,11 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
           if (j <= last0) {
             const int sv = j % C::kVStages;
-            ok = warp_wait_bar(bar(C::kBarPFull + 0), static_cast<uint32_t>(j & 1), wc) &&
-                 warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc);
+            ok = issue_pv(0, j, sv, split_p_tile(qt0, j));
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(0, j, sv, split_p_tile(qt0, j));
             if (j == last0) mma_commit_elect(bar(C::kBarOFinal + 0));
             if (j > last1 && j + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));
           }
@@ -447,39 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kTile; ++k) s[k] = (k <= lastcol) ? s[k] : fill;
       }
       // tile max of x = s * c: c * max(s) for c > 0, c * min(s) for c < 0 (exact under rounding)
-      float e0, e1, e2, e3;
-      if (c_pos) {
-        e0 = max3f(s[0], s[1], s[2]);
-        e1 = max3f(s[3], s[4], s[5]);
-        e2 = max3f(s[6], s[7], s[8]);
-        e3 = max3f(s[9], s[10], s[11]);
-#pragma unroll
-        for (int k = 12; k < kTile - 8; k += 8) {
-          e0 = max3f(e0, s[k], s[k + 1]);
-          e1 = max3f(e1, s[k + 2], s[k + 3]);
-          e2 = max3f(e2, s[k + 4], s[k + 5]);
-          e3 = max3f(e3, s[k + 6], s[k + 7]);
-        }
-        e0 = max3f(e0, s[kTile - 4], s[kTile - 3]);
-        e1 = max3f(e1, s[kTile - 2], s[kTile - 1]);
-        e0 = max3f(e0, e1, fmaxf(e2, e3));
-      } else {
-        e0 = min3f(s[0], s[1], s[2]);
-        e1 = min3f(s[3], s[4], s[5]);
-        e2 = min3f(s[6], s[7], s[8]);
-        e3 = min3f(s[9], s[10], s[11]);
-#pragma unroll
-        for (int k = 12; k < kTile - 8; k += 8) {
-          e0 = min3f(e0, s[k], s[k + 1]);
-          e1 = min3f(e1, s[k + 2], s[k + 3]);
-          e2 = min3f(e2, s[k + 4], s[k + 5]);
-          e3 = min3f(e3, s[k + 6], s[k + 7]);
-        }
-        e0 = min3f(e0, s[kTile - 4], s[kTile - 3]);
-        e1 = min3f(e1, s[kTile - 2], s[kTile - 1]);
-        e0 = min3f(e0, e1, fminf(e2, e3));
-      }
-      const float m_tile = e0 * c;
+      const float m_tile = (c_pos ? row_reduce<true>(s) : row_reduce<false>(s)) * c;
       const float m_new = fmaxf(m_used, m_tile);
       const bool rescale = m_new > m_used + kRescaleThreshold;  // always true on the first tile
       float alpha = 1.f;
@@ -488,34 +530,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum *= alpha;
         m_used = m_new;
       }
-      // P = 2^(s * c - m) over the first 64 columns of S_i (16-bit pairs);
-      // the tile with few-key rows also gets its rounding residual.
+      // O_i holds the sum up to tile j-1 under the old max; PV_i(j-1) has
+      // completed because S_i(j) was issued after it and has completed. TMEM
+      // access is warp-collective: the whole warp rescales, others by 1.
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) rescale_o<D>(o_col, alpha);
+      // P = 2^(s * c - m) over the first 64 columns of S_i, published in two
+      // halves (keys 0-63, 64-127) so the PV MMA can start on the first.
+      float psum;
       if (split_p_tile(qt, j)) {
-        l_sum += softmax_exp_store<FP16, true>(s, c, m_used, s_col);
+        psum = softmax_exp_half<FP16, true, 0>(s, c, m_used, s_col);
       } else {
-        l_sum += softmax_exp_store<FP16, false>(s, c, m_used, s_col);
-      }
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O_i holds the sum up to tile j-1 under the old max; PV_i(j-1) has
-        // completed because S_i(j) was issued after it and has completed.
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t o[32];
-          tmem_ld32(o_col + q * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float2 v = fmul2(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])),
-                                   make_float2(alpha, alpha));
-            o[k] = __float_as_uint(v.x);
-            o[k + 1] = __float_as_uint(v.y);
-          }
-          tmem_st32(o_col + q * 32, o);
-        }
+        psum = softmax_exp_half<FP16, false, 0>(s, c, m_used, s_col);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull + wg));
+      mbar_arrive(bar(C::kBarPFull + 2 * wg));
+      if (split_p_tile(qt, j)) {
+        psum += softmax_exp_half<FP16, true, 1>(s, c, m_used, s_col);
+      } else {
+        psum += softmax_exp_half<FP16, false, 1>(s, c, m_used, s_col);
+      }
+      l_sum += psum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + 2 * wg + 1));
     }
     if (last >= 0 && ok) ok = warp_wait_bar(bar(C::kBarOFinal + wg), 0, wc);
     if (last >= 0 && ok) {
