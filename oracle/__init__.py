@@ -60,6 +60,9 @@ def _load():
         lib.oracle_attention_rows.restype = ctypes.c_int
         lib.oracle_tiled_reference.argtypes = common + [i64, f64p, f64p]
         lib.oracle_tiled_reference.restype = ctypes.c_int
+        lib.oracle_attention_varlen.argtypes = [u16p, u16p, u16p, i64p, i64p, i64, i64, i64, i64, ctypes.c_double,
+                                                ctypes.c_int, ctypes.c_int, f64p, f64p, ctypes.c_int]
+        lib.oracle_attention_varlen.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -131,6 +134,34 @@ def attention_rows(q, k, v, scale: float, causal: bool, dtype: str, rows, nthrea
         _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double), int(nthreads or default_threads()))
     if rc:
         raise ValueError(f"oracle_attention_rows failed ({rc})")
+    return o, lse
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool, dtype: str, nthreads: int | None = None):
+    """Packed sequences with grouped-query heads and bottom-right causal alignment.
+
+    q: [total_q, Hq, D], k and v: [total_k, Hkv, D] (uint16 patterns); cu_q, cu_k: B+1
+    prefix offsets. Returns (O [total_q, Hq, D] float64, LSE [Hq, total_q] float64);
+    a query with no visible key has O = 0 and LSE = -inf.
+    """
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    if q.ndim != 3 or k.ndim != 3 or k.shape != v.shape or q.shape[2] != k.shape[2]:
+        raise ValueError("q must be [total_q, Hq, D], k and v [total_k, Hkv, D]")
+    cu_q = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int64))
+    cu_k = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int64))
+    B = len(cu_q) - 1
+    if len(cu_k) != B + 1 or cu_q[-1] != q.shape[0] or cu_k[-1] != k.shape[0]:
+        raise ValueError("cu_seqlens do not match the tensors")
+    total_q, Hq, D = q.shape
+    Hkv = k.shape[1]
+    o = np.empty((total_q, Hq, D), dtype=np.float64)
+    lse = np.empty((Hq, total_q), dtype=np.float64)
+    rc = _load().oracle_attention_varlen(
+        _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16), _ptr(cu_q, ctypes.c_int64),
+        _ptr(cu_k, ctypes.c_int64), B, Hq, Hkv, D, float(scale), int(bool(causal)), DTYPE_CODES[dtype],
+        _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double), int(nthreads or default_threads()))
+    if rc:
+        raise ValueError(f"oracle_attention_varlen failed ({rc})")
     return o, lse
 
 

@@ -38,6 +38,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <limits>
 #include <thread>
@@ -221,6 +222,63 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
         for (int64_t d = 0; d < D; ++d) Vvis[j * D + d] = decode(v[at(p, b, j, h, d)], dtype);
       }
       lse_rows[r] = finish_row(p, s.data(), nvis, Vvis, &o_rows[r * D]);
+    }
+  });
+  return 0;
+}
+
+// The definition for a batch of sequences packed without padding, with
+// grouped-query heads and queries and keys of different lengths:
+//   q, o : [total_q, Hq, D]; k, v : [total_k, Hkv, D]; lse : [Hq, total_q]
+//   sequence b owns query rows cu_q[b] .. cu_q[b+1]-1 and key rows
+//   cu_k[b] .. cu_k[b+1]-1 (nq and nk rows); query head h reads key/value head
+//   h / (Hq / Hkv);
+//   vis(i) = { j < nk : (j <= i + nk - nq if causal) }  (causal aligned at the
+//   bottom-right corner, which is the square mask when nq == nk);
+//   a query with no visible key has O = 0 and LSE = -inf (an empty sum).
+// Rows are computed one at a time with the same arithmetic as finish_row.
+int oracle_attention_varlen(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int64_t* cu_q,
+                            const int64_t* cu_k, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, double scale,
+                            int causal, int dtype, double* o, double* lse, int nthreads) {
+  if (!q || !k || !v || !cu_q || !cu_k || !o || !lse || B < 0 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv != 0 ||
+      (dtype != 0 && dtype != 1))
+    return 1;
+  for (int64_t b = 0; b < B; ++b)
+    if (cu_q[b + 1] < cu_q[b] || cu_k[b + 1] < cu_k[b] || cu_q[0] != 0 || cu_k[0] != 0) return 2;
+  const int64_t total_q = cu_q[B];
+  const int64_t group = Hq / Hkv;
+  // one task per (b, h, i)
+  std::vector<int64_t> task_b;
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = cu_q[b]; i < cu_q[b + 1]; ++i) task_b.push_back(b);
+  const int64_t n_rows = static_cast<int64_t>(task_b.size());
+  parallel_for(n_rows * Hq, nthreads, [&](int64_t lo, int64_t hi) {
+    std::vector<double> s, Vvis, qrow(static_cast<size_t>(D));
+    for (int64_t t = lo; t < hi; ++t) {
+      const int64_t row = t / Hq, h = t % Hq, b = task_b[row];
+      const int64_t nq = cu_q[b + 1] - cu_q[b], nk = cu_k[b + 1] - cu_k[b];
+      const int64_t i = row - cu_q[b];
+      const int64_t hk = h / group;
+      int64_t nvis = nk;
+      if (causal) nvis = std::min(nk, std::max<int64_t>(0, i + nk - nq + 1));
+      double* orow = &o[(row * Hq + h) * D];
+      if (nvis == 0) {
+        for (int64_t d = 0; d < D; ++d) orow[d] = 0.0;
+        lse[h * total_q + row] = -std::numeric_limits<double>::infinity();
+        continue;
+      }
+      for (int64_t d = 0; d < D; ++d) qrow[d] = decode(q[(row * Hq + h) * D + d], dtype);
+      s.assign(static_cast<size_t>(nvis), 0.0);
+      Vvis.assign(static_cast<size_t>(nvis * D), 0.0);
+      for (int64_t j = 0; j < nvis; ++j) {
+        const int64_t krow = cu_k[b] + j;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qrow[d] * decode(k[(krow * Hkv + hk) * D + d], dtype);
+        s[j] = scale * dot;
+        for (int64_t d = 0; d < D; ++d) Vvis[j * D + d] = decode(v[(krow * Hkv + hk) * D + d], dtype);
+      }
+      Problem p{q, k, v, 1, nk, 1, D, scale, causal, dtype};
+      lse[h * total_q + row] = finish_row(p, s.data(), nvis, Vvis, orow);
     }
   });
   return 0;
