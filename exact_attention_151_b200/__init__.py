@@ -16,7 +16,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_into", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
+__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
            "FA_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
 
@@ -31,7 +31,8 @@ FA_BF16 = 0
 FA_FP16 = 1
 
 # Every entry point declared in include/fa.h.
-EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_status_sync", "fa_fwd_debug")
+EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen",
+                    "fa_status_sync", "fa_fwd_debug")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -70,6 +71,11 @@ def load_library():
     lib.fa_fwd.restype = i32
     lib.fa_fwd_debug.argtypes = fwd_args + [ctypes.c_uint64, i32]
     lib.fa_fwd_debug.restype = i32
+    lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32, vp]
+    lib.fa_fwd_gqa.restype = i32
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32,
+                                  i32, vp]
+    lib.fa_fwd_varlen.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
     _lib = lib
@@ -115,20 +121,31 @@ def _dtype_code(t) -> int:
     raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
 
 
-def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, **debug) -> None:
-    """Run the forward into caller-provided ``o`` ([B,N,H,D]) and ``lse`` (fp32 [B,H,N])."""
-    import torch
-
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
-        raise ValueError("q, k, v, o must share one [B, N, H, D] shape")
-    B, N, H, D = q.shape
-    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
-        raise ValueError("lse must be float32 [B, H, N]")
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+def _check_cuda(**tensors):
+    for name, t in tensors.items():
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+
+
+def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, **debug) -> None:
+    """Forward into caller-provided ``o`` ([B,Nq,Hq,D]) and ``lse`` (fp32 [B,Hq,Nq]).
+
+    k and v may have their own length Nk and Hkv heads (Hq % Hkv == 0); with
+    causal=True the mask is aligned at the bottom-right corner.
+    """
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or o.shape != q.shape:
+        raise ValueError("q, o must be [B, Nq, Hq, D] and k, v [B, Nk, Hkv, D]")
+    B, Nq, Hq, D = q.shape
+    Bk, Nk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q and k/v disagree on batch or head dimension")
+    if tuple(lse.shape) != (B, Hq, Nq) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, Hq, Nq]")
+    _check_cuda(q=q, k=k, v=v, o=o, lse=lse)
     if k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
         raise TypeError("q, k, v and o must share one dtype")
     code = _dtype_code(q)
@@ -136,18 +153,61 @@ def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, 
         scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream(q.device).cuda_stream
     with torch.cuda.device(q.device):
-        st = fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, D,
-                     float(scale), causal, code, stream, **debug)
+        if Nk == Nq and Hkv == Hq:
+            st = fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Nq, Hq, D,
+                         float(scale), causal, code, stream, **debug)
+        else:
+            if debug:
+                raise ValueError("debug hooks exist only for Nq == Nk and Hq == Hkv")
+            st = load_library().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                           B, Nq, Nk, Hq, Hkv, D, ctypes.c_float(float(scale)), int(bool(causal)),
+                                           code, stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
 
 
 def fwd(q, k, v, scale: float | None = None, causal: bool = False):
-    """Exact attention forward. Returns (o [B,N,H,D] like q, lse float32 [B,H,N])."""
+    """Exact attention forward. Returns (o [B,Nq,Hq,D] like q, lse float32 [B,Hq,Nq])."""
     import torch
 
-    B, N, H, D = q.shape
+    B, Nq, Hq, D = q.shape
     o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     fwd_into(q, k, v, o, lse, scale=scale, causal=causal)
+    return o, lse
+
+
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, scale: float | None = None,
+               causal: bool = False, o=None, lse=None):
+    """Forward over packed sequences: q [total_q, Hq, D], k/v [total_k, Hkv, D],
+    cu_seqlens_* int32 CUDA tensors of B+1 offsets. Returns (o like q, lse fp32 [Hq, total_q]).
+    Inconsistent offsets are reported by status_sync() as FA_ERR_INVALID_ARG."""
+    import torch
+
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or q.shape[2] != k.shape[2]:
+        raise ValueError("q must be [total_q, Hq, D] and k, v [total_k, Hkv, D]")
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_k.shape != cu_seqlens_q.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must be 1-D with B+1 entries")
+    B = cu_seqlens_q.numel() - 1
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _check_cuda(q=q, k=k, v=v, o=o, lse=lse, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k)
+    if k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
+        raise TypeError("q, k, v and o must share one dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = load_library().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                          cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                                          total_q, total_k, Hq, Hkv, D, ctypes.c_float(float(scale)),
+                                          int(bool(causal)), _dtype_code(q), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
     return o, lse

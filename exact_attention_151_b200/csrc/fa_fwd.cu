@@ -64,15 +64,15 @@ fa_status load_encoder() {
   return st;
 }
 
-// [B, N, H, D] 16-bit tensor viewed as 4-D (D, H, N, B), box (64, 1, 128, 1), 128B swizzle.
-fa_status make_tmap(CUtensorMap* map, const void* base, int64_t B, int64_t N, int64_t H, int64_t D, bool fp16) {
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
-                              static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(H * D * 2),
-                                 static_cast<cuuint64_t>(N * H * D * 2)};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = g_encode(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+// A [rows, H, D] 16-bit tensor (a dense [B, N, H, D] tensor is B*N rows)
+// viewed as 3-D (D, H, rows), box (64, 1, 128), 128B swizzle; rows past the
+// end are zero-filled by TMA.
+fa_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t H, int64_t D, bool fp16) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(H * D * 2)};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -107,10 +107,16 @@ fa_status check_device(int* dev_out) {
   return di.checked == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
 }
 
+// Problem shape as the host sees it (dense when cu_q == nullptr).
+struct Shape {
+  const int* cu_q;
+  const int* cu_k;
+  int64_t B, Nq, Nk, total_q, total_k, max_nq, Hq, Hkv, D;
+};
+
 template <int D, bool FP16>
 fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, float* lse,
-                 int64_t B, int64_t N, int64_t H, float scale, int causal, cudaStream_t stream, uint64_t limit_ns,
-                 int withhold) {
+                 const Shape& sh, float scale, int causal, cudaStream_t stream, uint64_t limit_ns, int withhold) {
   using C = Cfg<D>;
   auto kernel = fa_fwd_kernel<D, FP16>;
   const unsigned bit = 1u << ((D == 128 ? 2 : 0) + (FP16 ? 1 : 0));
@@ -145,11 +151,17 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   Params prm;
   prm.out = static_cast<uint16_t*>(o);
   prm.lse = lse;
-  prm.N = static_cast<int>(N);
-  prm.H = static_cast<int>(H);
-  prm.BH = static_cast<int>(B * H);
-  prm.n_tiles = static_cast<int>((N + kTile - 1) / kTile);
-  prm.n_blocks = static_cast<int>((N + kBlockRows - 1) / kBlockRows);
+  prm.cu_q = sh.cu_q;
+  prm.cu_k = sh.cu_k;
+  prm.Nq = static_cast<int>(sh.Nq);
+  prm.Nk = static_cast<int>(sh.Nk);
+  prm.total_q = static_cast<int>(sh.total_q);
+  prm.total_k = static_cast<int>(sh.total_k);
+  prm.Hq = static_cast<int>(sh.Hq);
+  prm.Hkv = static_cast<int>(sh.Hkv);
+  prm.BH = static_cast<int>(sh.B * sh.Hq);
+  prm.max_nq = static_cast<int>(sh.max_nq);
+  prm.n_blocks = static_cast<int>((sh.max_nq + kBlockRows - 1) / kBlockRows);
   // Softmax runs in base 2: x = s * scale * log2(e). A zero (or subnormal)
   // factor is replaced by +-FLT_MIN: every weight then still rounds to
   // exactly 1 (|s| < 2^40 for 16-bit inputs) while masked keys keep weight 0.
@@ -159,7 +171,7 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.causal = causal ? 1 : 0;
   prm.wait_limit_ns = static_cast<unsigned long long>(limit_ns);
   prm.withhold_v_load = withhold;
-  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * B * H;
+  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * sh.B * sh.Hq;
   kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -168,49 +180,68 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     return FA_ERR_CUDA;
   }
   if (debug_enabled()) {
-    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld N=%lld H=%lld causal=%d grid=%lld smem=%d\n", D,
-                 FP16 ? "fp16" : "bf16", (long long)B, (long long)N, (long long)H, causal, (long long)grid,
-                 C::kSmemBytes);
+    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d grid=%lld smem=%d\n",
+                 D, FP16 ? "fp16" : "bf16", (long long)sh.B, (long long)sh.Nq, (long long)sh.Nk, (long long)sh.Hq,
+                 (long long)sh.Hkv, sh.cu_q ? "packed" : "dense", causal, (long long)grid, C::kSmemBytes);
   }
   return FA_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N, int64_t H,
-                   int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream, uint64_t limit_ns,
-                   int withhold) {
-  if (B < 0 || N < 0 || H < 0) return FA_ERR_INVALID_ARG;
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& sh, float scale,
+                   int causal, fa_dtype dtype, fa_stream_t stream, uint64_t limit_ns, int withhold) {
+  if (sh.B < 0 || sh.Nq < 0 || sh.Nk < 0 || sh.Hq < 0 || sh.Hkv < 0 || sh.total_q < 0 || sh.total_k < 0 ||
+      sh.max_nq < 0)
+    return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (B == 0 || N == 0 || H == 0) return FA_OK;
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-  // int32 kernel indexing and TMA coordinate limits
-  const int64_t n_blocks = (N + kBlockRows - 1) / kBlockRows;
-  if (N > INT32_MAX || H > INT32_MAX || B > INT32_MAX) return FA_ERR_UNSUPPORTED;
-  if (B * H > INT32_MAX / n_blocks) return FA_ERR_UNSUPPORTED;
-  if (B * N > INT32_MAX / H) return FA_ERR_UNSUPPORTED;  // (b*N + i) * H + h fits int64 with room; keep rows int32
-  if ((static_cast<double>(B) * N * H * D * 2) >= 1099511627776.0) return FA_ERR_UNSUPPORTED;  // < 2^40 B
+  if (sh.Hq > 0 && (sh.Hkv < 1 || sh.Hq % sh.Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (sh.D != 64 && sh.D != 128) return FA_ERR_UNSUPPORTED;
+  if (sh.B == 0 || sh.Hq == 0 || sh.total_q == 0 || sh.max_nq == 0) return FA_OK;
+  if (!q || !o || !lse || (sh.total_k > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (sh.cu_q && !sh.cu_k) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (sh.total_k > 0 && (!aligned16(k) || !aligned16(v))))
+    return FA_ERR_MISALIGNED;
+  // int32 kernel indexing, TMA coordinate and tensor-size limits
+  const int64_t n_blocks = (sh.max_nq + kBlockRows - 1) / kBlockRows;
+  if (sh.total_q > INT32_MAX - 2 * kBlockRows || sh.total_k > INT32_MAX - 2 * kBlockRows || sh.Hq > INT32_MAX ||
+      sh.B > INT32_MAX || sh.max_nq > INT32_MAX - 2 * kBlockRows)
+    return FA_ERR_UNSUPPORTED;
+  if (sh.B * sh.Hq > INT32_MAX / n_blocks) return FA_ERR_UNSUPPORTED;
+  if (static_cast<double>(sh.total_q) * sh.Hq * sh.D * 2 >= 1099511627776.0 ||
+      static_cast<double>(sh.total_k) * sh.Hkv * sh.D * 2 >= 1099511627776.0)
+    return FA_ERR_UNSUPPORTED;  // each tensor < 2^40 bytes
   int dev = 0;
   fa_status st = check_device(&dev);
   if (st != FA_OK) return st;
   st = load_encoder();
   if (st != FA_OK) return st;
   const bool fp16 = dtype == FA_FP16;
+  // With no keys at all nothing is ever loaded from K or V; the maps only need
+  // a valid, aligned base.
+  const void* kb = sh.total_k > 0 ? k : q;
+  const void* vb = sh.total_k > 0 ? v : q;
+  const int64_t krows = sh.total_k > 0 ? sh.total_k : 1;
+  const int64_t khead = sh.total_k > 0 ? sh.Hkv : 1;
   CUtensorMap tq, tk, tv;
-  if (make_tmap(&tq, q, B, N, H, D, fp16) != FA_OK || make_tmap(&tk, k, B, N, H, D, fp16) != FA_OK ||
-      make_tmap(&tv, v, B, N, H, D, fp16) != FA_OK)
+  if (make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16) != FA_OK || make_tmap(&tk, kb, krows, khead, sh.D, fp16) != FA_OK ||
+      make_tmap(&tv, vb, krows, khead, sh.D, fp16) != FA_OK)
     return FA_ERR_CUDA;
   if (limit_ns == 0) limit_ns = kDefaultWaitLimitNs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128) {
-    return fp16 ? launch<128, true>(dev, tq, tk, tv, o, lse, B, N, H, scale, causal, s, limit_ns, withhold)
-                : launch<128, false>(dev, tq, tk, tv, o, lse, B, N, H, scale, causal, s, limit_ns, withhold);
+  if (sh.D == 128) {
+    return fp16 ? launch<128, true>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold)
+                : launch<128, false>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold);
   }
-  return fp16 ? launch<64, true>(dev, tq, tk, tv, o, lse, B, N, H, scale, causal, s, limit_ns, withhold)
-              : launch<64, false>(dev, tq, tk, tv, o, lse, B, N, H, scale, causal, s, limit_ns, withhold);
+  return fp16 ? launch<64, true>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold)
+              : launch<64, false>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold);
+}
+
+Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D) {
+  Shape sh{nullptr, nullptr, B, Nq, Nk, B * Nq, B * Nk, Nq, Hq, Hkv, D};
+  if (B < 0 || Nq < 0 || Nk < 0) sh.B = -1;  // rejected by fwd_impl
+  return sh;
 }
 
 }  // namespace
@@ -235,7 +266,30 @@ const char* fa_status_string(fa_status s) {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N, int64_t H,
                  int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
   try {
-    return fa::fwd_impl(q, k, v, o, lse, B, N, H, D, scale, causal, dtype, stream, 0, 0);
+    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream, 0, 0);
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t Nq,
+                     int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                     fa_stream_t stream) {
+  try {
+    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, Nq, Nk, Hq, Hkv, D), scale, causal, dtype, stream, 0, 0);
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int64_t B, int64_t max_seqlen_q, int64_t total_q, int64_t total_k,
+                        int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream) {
+  try {
+    if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+    fa::Shape sh{cu_seqlens_q, cu_seqlens_k, B, 0, 0, total_q, total_k, max_seqlen_q, Hq, Hkv, D};
+    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -245,8 +299,8 @@ fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, flo
                        int64_t H, int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream,
                        uint64_t wait_limit_ns, int withhold_v_load) {
   try {
-    return fa::fwd_impl(q, k, v, o, lse, B, N, H, D, scale, causal, dtype, stream, wait_limit_ns,
-                        withhold_v_load ? 1 : 0);
+    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream,
+                        wait_limit_ns, withhold_v_load ? 1 : 0);
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -266,12 +320,13 @@ fa_status fa_status_sync(fa_stream_t stream) {
   }
   if (word != 0) {
     const unsigned int zero = 0;
+    const fa_status which = (word & 1u) ? FA_ERR_TIMEOUT : FA_ERR_INVALID_ARG;
     if (cudaMemcpyToSymbolAsync(fa::g_status_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_CUDA;
     }
-    return FA_ERR_TIMEOUT;
+    return which;
   }
   return FA_OK;
 }

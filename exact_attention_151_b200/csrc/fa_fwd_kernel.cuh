@@ -64,8 +64,8 @@ constexpr int kLoadWarp = 9;      // warps 10 and 11 only keep warpgroup 2 whole
 // and the two softmax warpgroups take them. The shares must not exceed the
 // launch pool, or the increase would wait forever:
 constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 216;
-constexpr uint32_t kControlRegs = 72;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kControlRegs = 88;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.693147180559945309f;
@@ -141,12 +141,16 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Wai
 }
 
 // Tile (query tile qt, key tile j) whose P is applied as P16 + (P - P16).
-// Only the first key tile of the first query tile holds rows that see few
-// keys (causal rows 0..127, or every row when N <= 128); there a single
-// 16-bit rounding of P would weigh on the result about as much as the final
-// rounding of O, so the residual is added with a second MMA pass. Elsewhere
-// every row averages over more than 128 keys and the residual is negligible.
-__device__ __forceinline__ bool split_p_tile(int qt, int j) { return qt == 0 && j == 0; }
+// Rows that see at most 128 keys keep all of them in key tile 0; for such
+// rows a single 16-bit rounding of P weighs on the result about as much as
+// the final rounding of O, so the residual is added with a second MMA pass.
+// Causal: row i sees i + delta + 1 keys, so the tiles with such rows are those
+// starting at or before row 127 - delta; otherwise it is every tile when the
+// sequence has at most 128 keys. Elsewhere each row averages over more than
+// 128 keys and the residual is negligible.
+__device__ __forceinline__ bool split_p_tile(int qt, int j, int causal, int delta, int nk) {
+  return j == 0 && (causal ? (qt * kTile <= kTile - 1 - delta) : (nk <= kTile));
+}
 
 // Pairs of score columns whose exp2 runs on the FMA pipe instead of the
 // MUFU unit (every fourth pair): the two softmax warpgroups share each SM
@@ -236,14 +240,18 @@ __device__ __forceinline__ void rescale_o(uint32_t o_col, float alpha) {
 
 // Problem description passed by value.
 struct Params {
-  uint16_t* out;
-  float* lse;
-  int N, H;
-  int BH;        // B * H
-  int n_tiles;   // ceil(N / 128)
-  int n_blocks;  // ceil(N / 256)
+  uint16_t* out;        // [total_q, Hq, D]
+  float* lse;           // dense: [B, Hq, Nq]; packed: [Hq, total_q]
+  const int* cu_q;      // packed sequences: B+1 query row offsets (device memory); dense: null
+  const int* cu_k;      // packed sequences: B+1 key row offsets
+  int Nq, Nk;           // dense sequence lengths
+  int total_q, total_k; // rows of q/o and of k/v
+  int Hq, Hkv;          // query heads, key/value heads (Hq % Hkv == 0)
+  int BH;               // B * Hq
+  int max_nq;           // upper bound of every query length (sizes the grid)
+  int n_blocks;         // ceil(max_nq / 256)
   float scale_log2;
-  int causal;
+  int causal;           // key j visible to query i iff j <= i + nk - nq (bottom-right aligned)
   unsigned long long wait_limit_ns;
   int withhold_v_load;
 };
@@ -265,7 +273,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int N = prm.N;
   const int causal = prm.causal;
 
   int bh, level;
@@ -295,14 +302,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     level = static_cast<int>(blockIdx.x) % prm.n_blocks;
   }
   const int mb = causal ? (prm.n_blocks - 1 - level) : level;
-  const int b = bh / prm.H;
-  const int h = bh % prm.H;
+  const int b = bh / prm.Hq;
+  const int h = bh % prm.Hq;
+  const int hk = h / (prm.Hq / prm.Hkv);  // key/value head of this query head
+  // This sequence's rows: queries q0 .. q0+nq-1, keys k0 .. k0+nk-1.
+  int q0, nq, k0, nk;
+  if (prm.cu_q != nullptr) {
+    q0 = prm.cu_q[b];
+    nq = prm.cu_q[b + 1] - q0;
+    k0 = prm.cu_k[b];
+    nk = prm.cu_k[b + 1] - k0;
+    const bool bad = q0 < 0 || nq < 0 || nq > prm.max_nq || static_cast<int64_t>(q0) + nq > prm.total_q || k0 < 0 ||
+                     nk < 0 || static_cast<int64_t>(k0) + nk > prm.total_k;
+    if (bad) {  // inconsistent offsets: report, touch nothing
+      if (threadIdx.x == 0) atomicOr(&g_status_word, 2u);
+      return;
+    }
+  } else {
+    q0 = b * prm.Nq;
+    nq = prm.Nq;
+    k0 = b * prm.Nk;
+    nk = prm.Nk;
+  }
+  if (mb * kBlockRows >= nq) return;  // block past the end of this sequence
+  const int n_qt = (nq + kTile - 1) / kTile;
+  const int n_kt = (nk + kTile - 1) / kTile;
+  const int delta = nk - nq;  // causal offset: query i sees keys j <= i + delta
   const int qt0 = 2 * mb;
   const int qt1 = 2 * mb + 1;
-  const bool q1_valid = qt1 < prm.n_tiles;
-  // key tiles visited, and the last key tile of each query tile
-  const int last0 = causal ? qt0 : prm.n_tiles - 1;
-  const int last1 = q1_valid ? (causal ? qt1 : prm.n_tiles - 1) : -1;
+  const bool q1_valid = qt1 < n_qt;
+  // last key tile holding a key visible to some row of query tile qt (-1: none)
+  auto last_key_tile = [&](int qt) -> int {
+    if (nk == 0) return -1;
+    if (!causal) return n_kt - 1;
+    const int last_key = qt * kTile + kTile - 1 + delta;
+    if (last_key < 0) return -1;
+    return min(n_kt - 1, last_key / kTile);
+  };
+  const int last0 = last_key_tile(qt0);
+  const int last1 = q1_valid ? last_key_tile(qt1) : -1;
   const int n_kv = (last1 > last0 ? last1 : last0) + 1;
 
   if (threadIdx.x == 0) {
@@ -351,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx_elect(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
       for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, (qt0 + i) * kTile, b, bar(C::kBarQ));
+          tma_load_3d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0 + (qt0 + i) * kTile, bar(C::kBarQ));
       const bool withhold = prm.withhold_v_load && blockIdx.x == 0;
       int nk = 0, nv = 0;  // K and V tiles issued
       for (int j = 0; j < n_kv; ++j) {
@@ -361,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, j * kTile, b, bar(C::kBarKFull + sk));
+          tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, k0 + j * kTile, bar(C::kBarKFull + sk));
         nk = j + 1;
         const int sv = j % C::kVStages;
         if (j >= C::kVStages &&
@@ -370,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(withhold && j == 0)) {
           mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
           for (int hf = 0; hf < C::kHalves; ++hf)
-            tma_load_4d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, j * kTile, b, bar(C::kBarVFull + sv));
+            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, k0 + j * kTile, bar(C::kBarVFull + sv));
         }
         nv = j + 1;
       }
@@ -447,6 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv_half(i, j, sv, split, 1);
         return true;
       };
+      const bool split0 = split_p_tile(qt0, 0, causal, delta, nk);
+      const bool split1 = split_p_tile(qt1, 0, causal, delta, nk);
       bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
       for (int j = 0; ok && j <= n_kv; ++j) {
         const int sk = j % C::kKStages;
@@ -459,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1 && j - 1 <= last1) {
           // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
           const int jp = j - 1, sv = jp % C::kVStages;
-          ok = issue_pv(1, jp, sv, split_p_tile(qt1, jp));
+          ok = issue_pv(1, jp, sv, split1 && jp == 0);
           if (!ok) break;
           if (jp == last1) mma_commit_elect(bar(C::kBarOFinal + 1));
           if (jp + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
@@ -469,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
           if (j <= last0) {
             const int sv = j % C::kVStages;
-            ok = issue_pv(0, j, sv, split_p_tile(qt0, j));
+            ok = issue_pv(0, j, sv, split0 && j == 0);
             if (!ok) break;
             if (j == last0) mma_commit_elect(bar(C::kBarOFinal + 0));
             if (j > last1 && j + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));
@@ -515,8 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kTile; ++k) s[k] = __uint_as_float(r[k / 32][k % 32]);
       }
       const int kbase = j * kTile;
-      if ((causal && j == qt) || kbase + kTile > N) {
-        const int lastcol = (causal ? min(N - 1, qi) : (N - 1)) - kbase;  // last visible column
+      if (kbase + kTile > nk || (causal && kbase + kTile - 1 > qt * kTile + delta)) {
+        // last visible column of this row in this tile (may be < 0: none)
+        const int lastcol = (causal ? min(nk - 1, qi + delta) : (nk - 1)) - kbase;
 #pragma unroll
         for (int k = 0; k < kTile; ++k) s[k] = (k <= lastcol) ? s[k] : fill;
       }
@@ -537,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(s * c - m) over the first 64 columns of S_i, published in two
       // halves (keys 0-63, 64-127) so the PV MMA can start on the first.
       float psum;
-      if (split_p_tile(qt, j)) {
+      if (split_p_tile(qt, j, causal, delta, nk)) {
         psum = softmax_exp_half<FP16, true, 0>(s, c, m_used, s_col);
       } else {
         psum = softmax_exp_half<FP16, false, 0>(s, c, m_used, s_col);
@@ -545,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + 2 * wg));
-      if (split_p_tile(qt, j)) {
+      if (split_p_tile(qt, j, causal, delta, nk)) {
         psum += softmax_exp_half<FP16, true, 1>(s, c, m_used, s_col);
       } else {
         psum += softmax_exp_half<FP16, false, 1>(s, c, m_used, s_col);
@@ -556,11 +597,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(C::kBarPFull + 2 * wg + 1));
     }
     if (last >= 0 && ok) ok = warp_wait_bar(bar(C::kBarOFinal + wg), 0, wc);
+    // Epilogue. A row with no visible key (bottom-right causal with nq > nk,
+    // or nk == 0) gets O = 0 and LSE = -inf, whatever its TMEM lanes hold.
+    const bool row_valid = (wg == 0 || q1_valid) && qi < nq;
+    const bool row_has_keys = nk > 0 && (!causal || qi + delta >= 0);
+    uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + h) * D;
+    float* lse_at = prm.lse + (prm.cu_q != nullptr
+                                   ? static_cast<int64_t>(h) * prm.total_q + q0 + qi
+                                   : (static_cast<int64_t>(b) * prm.Hq + h) * prm.Nq + qi);
     if (last >= 0 && ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l_sum;
-      const bool row_valid = qi < N;
-      uint16_t* orow = prm.out + ((static_cast<int64_t>(b) * N + qi) * prm.H + h) * D;
+      const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
@@ -571,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 16; ++k) {
           const float2 v = fmul2(make_float2(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1])),
                                  make_float2(inv_l, inv_l));
-          pk[k] = pack2<FP16>(v.x, v.y);
+          pk[k] = row_has_keys ? pack2<FP16>(v.x, v.y) : 0u;
         }
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
@@ -579,7 +626,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (row_valid) prm.lse[(static_cast<int64_t>(b) * prm.H + h) * N + qi] = (m_used + lg2_approx(l_sum)) * kLn2;
+      if (row_valid) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+    } else if (last < 0 && row_valid) {
+      // no key tile at all for this query tile
+      uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+      for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+      *lse_at = -INFINITY;
     }
   }
 

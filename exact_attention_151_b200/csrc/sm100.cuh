@@ -226,6 +226,18 @@ __device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const void* tmap
       : "memory");
 }
 
+// 3-D tiled tensor load, issued by one elected lane of a converged warp.
+__device__ __forceinline__ void tma_load_3d_elect(uint32_t dst, const void* tmap, int c0, int c1, int c2,
+                                                  uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {

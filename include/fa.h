@@ -58,8 +58,8 @@ typedef enum {
   FA_ERR_TIMEOUT = 5      /* a device-side wait ran out (reported by fa_status_sync) */
 } fa_status;
 
-/* Limits checked before launch: 1 <= D in {64,128}; B*H <= 2^31-1;
- * N <= 2^31-1; each of q/k/v/o spans < 2^40 bytes. */
+/* Limits checked before launch: D in {64,128}; B*H*ceil(N/256) <= 2^31-1;
+ * rows (B*N, or total) below 2^31 - 512; each of q/k/v/o spans < 2^40 bytes. */
 
 /* Static, human-readable name of a status code; never NULL. */
 const char* fa_status_string(fa_status status);
@@ -89,10 +89,55 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int64_t H, int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * fa_fwd_gqa - fa_fwd generalised to grouped-query heads and to queries and
+ * keys of different lengths (cross-attention); fa_fwd(..., N, H, ...) is
+ * fa_fwd_gqa(..., Nq = Nk = N, Hq = Hkv = H, ...).
+ *
+ *   q, o   : [B, Nq, Hq,  D] contiguous          k, v : [B, Nk, Hkv, D] contiguous
+ *   lse    : float32 [B, Hq, Nq]
+ *   Hq % Hkv == 0; query head h reads key/value head h / (Hq / Hkv)
+ *     (grouped-query / multi-query attention: llmtrend.com FlashAttention
+ *     page, Mistral case; separate query and key lengths: the same page's
+ *     limitations section, cross-attention).
+ *   causal : key j visible to query i iff j <= i + (Nk - Nq), i.e. the mask is
+ *            aligned at the bottom-right corner (the square mask when Nq == Nk).
+ *            A query with no visible key (possible when Nq > Nk) gets O = 0 and
+ *            LSE = -inf; so does every query when Nk == 0.
+ * Errors and asynchrony as fa_fwd; Hkv < 1 or Hq % Hkv != 0 -> FA_ERR_INVALID_ARG.
+ */
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t Nq,
+                     int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                     fa_stream_t stream);
+
+/*
+ * fa_fwd_varlen - forward over B sequences of different lengths packed
+ * without padding (the padding-free form of the pages' padding mask,
+ * jsqmd.com page, usage notes), with grouped-query heads.
+ *
+ *   q, o          : [total_q, Hq,  D] contiguous; sequence b owns query rows
+ *                   cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *   k, v          : [total_k, Hkv, D] contiguous; key rows cu_seqlens_k[b] ..
+ *   cu_seqlens_q/k: int32 DEVICE arrays of B+1 non-decreasing offsets,
+ *                   cu[0] = 0, cu[B] = total_q / total_k
+ *   max_seqlen_q  : >= every query length (sizes the grid)
+ *   lse           : float32 [Hq, total_q]
+ *   causal, GQA, empty rows: as fa_fwd_gqa, per sequence (nq, nk its lengths).
+ * The offsets live in device memory and are checked by the kernel: a sequence
+ * whose offsets are inconsistent (decreasing, beyond total, or longer than
+ * max_seqlen_q) is skipped, its outputs are left untouched, and
+ * fa_status_sync reports FA_ERR_INVALID_ARG.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int64_t B, int64_t max_seqlen_q, int64_t total_q, int64_t total_k,
+                        int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream);
+
+/*
  * fa_status_sync - synchronise `stream`, then read and clear this device's
- * status word. Returns FA_OK, FA_ERR_TIMEOUT if a kernel on this device gave
- * up on a bounded wait since the last call (its outputs are then invalid),
- * or FA_ERR_CUDA if the synchronisation itself failed.
+ * status word. Returns FA_OK; FA_ERR_TIMEOUT if a kernel on this device gave
+ * up on a bounded wait since the last call (its outputs are then invalid);
+ * FA_ERR_INVALID_ARG if fa_fwd_varlen met inconsistent sequence offsets; or
+ * FA_ERR_CUDA if the synchronisation itself failed.
  */
 fa_status fa_status_sync(fa_stream_t stream);
 

@@ -57,3 +57,25 @@ def test_bad_dtype_and_scale():
     assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, 0.125, False, 7, 0) == fa.FA_ERR_INVALID_ARG
     assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, float("inf"), False, fa.FA_BF16, 0) == fa.FA_ERR_INVALID_ARG
     assert fa.fwd_ptr(P, P, P, P, P, 1, 16, 1, 64, float("nan"), True, fa.FA_FP16, 0) == fa.FA_ERR_INVALID_ARG
+
+
+def test_general_entry_points_validate_before_any_device_call():
+    lib = fa.load_library()
+    f32 = __import__("ctypes").c_float
+    # Hq not a multiple of Hkv
+    assert lib.fa_fwd_gqa(P, P, P, P, P, 1, 16, 32, 6, 4, 64, f32(0.1), 0, fa.FA_BF16, 0) == fa.FA_ERR_INVALID_ARG
+    # no key/value heads
+    assert lib.fa_fwd_gqa(P, P, P, P, P, 1, 16, 32, 6, 0, 64, f32(0.1), 0, fa.FA_BF16, 0) == fa.FA_ERR_INVALID_ARG
+    # negative key length
+    assert lib.fa_fwd_gqa(P, P, P, P, P, 1, 16, -1, 4, 4, 64, f32(0.1), 0, fa.FA_BF16, 0) == fa.FA_ERR_INVALID_ARG
+    # empty query side is a no-op
+    assert lib.fa_fwd_gqa(0, 0, 0, 0, 0, 1, 0, 32, 4, 4, 64, f32(0.1), 0, fa.FA_BF16, 0) == fa.FA_OK
+    # varlen without offsets
+    assert lib.fa_fwd_varlen(P, P, P, P, P, 0, 0, 2, 16, 32, 32, 4, 4, 64, f32(0.1), 0, fa.FA_BF16, 0) == \
+        fa.FA_ERR_INVALID_ARG
+    # varlen with misaligned output
+    assert lib.fa_fwd_varlen(P, P, P, P + 2, P, P, P, 2, 16, 32, 32, 4, 4, 64, f32(0.1), 0, fa.FA_BF16, 0) == \
+        fa.FA_ERR_MISALIGNED
+    # varlen head dim not supported
+    assert lib.fa_fwd_varlen(P, P, P, P, P, P, P, 2, 16, 32, 32, 4, 4, 96, f32(0.1), 0, fa.FA_BF16, 0) == \
+        fa.FA_ERR_UNSUPPORTED
