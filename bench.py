@@ -63,6 +63,14 @@ def measured_peak():
         return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
 
 
+def measured_hbm() -> float:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"])
+    except Exception:
+        return 6650.0
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
     try:
@@ -144,8 +152,16 @@ def row_flops(w, rows) -> float:
     import numpy as np
 
     rows = np.asarray(rows)
-    nvis = (rows[:, 2] + 1) if w.causal else np.full(len(rows), w.N)
+    nk, nq = w.n_keys, w.N
+    if w.causal:
+        nvis = np.clip(rows[:, 2] + nk - nq + 1, 0, nk)
+    else:
+        nvis = np.full(len(rows), nk)
     return float(4.0 * w.D * nvis.sum())
+
+
+def is_square(w) -> bool:
+    return w.n_keys == w.N and w.kv_heads == w.H
 
 
 def oracle_row_sample(w, q, k, v, target_s: float, seed: int = 0):
@@ -158,6 +174,19 @@ def oracle_row_sample(w, q, k, v, target_s: float, seed: int = 0):
     Q, K, V = bits(q), bits(k), bits(v)
     rng = np.random.default_rng(seed)
     threads = oracle.default_threads()
+    if not is_square(w):
+        # decode-like shapes: the whole (small) query side through the packed form
+        B, Nq, Hq, D = q.shape
+        Nk, Hkv = k.shape[1], k.shape[2]
+        t0 = time.perf_counter()
+        o, lse = oracle.attention_varlen(Q.reshape(B * Nq, Hq, D), K.reshape(B * Nk, Hkv, D), V.reshape(B * Nk, Hkv, D),
+                                         np.arange(B + 1) * Nq, np.arange(B + 1) * Nk, w.softmax_scale, w.causal,
+                                         w.dtype, nthreads=threads)
+        dt = time.perf_counter() - t0
+        rows = np.array([(b, h, i) for b in range(B) for h in range(Hq) for i in range(Nq)], dtype=np.int64)
+        o_rows = o.reshape(B, Nq, Hq, D)[rows[:, 0], rows[:, 2], rows[:, 1]]
+        lse_rows = lse.reshape(Hq, B, Nq)[rows[:, 1], rows[:, 0], rows[:, 2]]
+        return rows, o_rows, lse_rows, dt, threads
 
     def draw(n):
         return np.stack([rng.integers(0, w.B, n), rng.integers(0, w.H, n), rng.integers(0, w.N, n)], axis=1)
@@ -207,10 +236,13 @@ def run_reference(args, w):
 
 
 def workload_config(w):
-    return {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "dtype": w.dtype, "causal": w.causal,
+    extra = {} if is_square(w) else {"Nk": w.n_keys, "Hkv": w.kv_heads, "causal_alignment": "bottom-right"}
+    if w.splitkv:
+        extra["path"] = "split-KV (fa_fwd_splitkv: partial kernel + merge kernel)"
+    return {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "dtype": w.dtype, "causal": w.causal, **extra,
             "scale": w.softmax_scale, "flops_per_step": w.flops, "seed": w.seed,
             "inputs": f"Q~N(0,{w.q_std}^2) K~N(0,{w.k_std}^2) V~{'U(-1,1)' if w.v_dist == 'uniform' else 'N(0,1)'}",
-            "l2": "no flush: Q+K+V+O exceed the 126 MB L2" if 8 * w.B * w.N * w.H * w.D > 126e6 else
+            "l2": "no flush: Q+K+V+O exceed the 126 MB L2" if w.min_hbm_bytes > 126e6 else
                   "L2 flushed between steps (256 MiB write, outside the per-step kernel events)"}
 
 
@@ -257,12 +289,20 @@ def main():
     od = torch.empty_like(qd)
     lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     flush = None
-    if 8 * w.B * w.N * w.H * w.D <= 126e6:
+    if w.min_hbm_bytes <= 126e6:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    kernels_per_step = 1
+    if w.splitkv:
+        n_splits, ws_bytes = fa.splitkv_plan(w.B, w.N, w.n_keys, w.H, w.D)
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        kernels_per_step = 2 if n_splits > 1 else 1
 
     def step():
-        fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
+        if w.splitkv:
+            fa.fwd_splitkv(qd, kd, vd, scale=w.softmax_scale, causal=w.causal, workspace=workspace, o=od, lse=lsed)
+        else:
+            fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
 
     for _ in range(args.warmup):
         step()
@@ -313,7 +353,7 @@ def main():
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
+        step()
         oh.copy_(od, non_blocking=True)
         lseh.copy_(lsed, non_blocking=True)
 
@@ -332,28 +372,37 @@ def main():
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
     e2e_value = w.flops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
-    h2d = 3 * q.numel() * q.element_size()
+    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     d2h = q.numel() * q.element_size() + lseh.numel() * 4
 
     if rank == 0:
         peak, peak_sus, peak_src = measured_peak()
         achieved = w.flops / (avg_launch_ms * 1e-3) / 1e12
         traffic, traffic_how = recorded_traffic(w.name)
+        intensity = w.flops / w.min_hbm_bytes
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": workload_config(w),
             "pct_of_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
-                         "frac_of_sustained_peak": achieved / peak_sus,
-                         "algorithmic_bytes": w.min_hbm_bytes,
-                         "traffic_source": traffic_how},
+            "roofline": ({"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                          "frac": achieved / peak, "traffic": traffic,
+                          "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
+                          "frac_of_sustained_peak": achieved / peak_sus,
+                          "algorithmic_bytes": w.min_hbm_bytes,
+                          "traffic_source": traffic_how}
+                         if intensity >= 300 else
+                         {"bound": "hbm", "achieved": w.min_hbm_bytes / (avg_launch_ms * 1e-3) / 1e9,
+                          "peak": measured_hbm(), "unit": "GB/s",
+                          "frac": w.min_hbm_bytes / (avg_launch_ms * 1e-3) / 1e9 / measured_hbm(),
+                          "traffic": traffic, "algorithmic_bytes": w.min_hbm_bytes,
+                          "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                          "arithmetic_intensity_flop_per_byte": intensity,
+                          "note": "per-step time covers the attention kernel and the split merge kernel"}),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "clocks": clocks.summary(),
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * kernels_per_step,
             "kernel_source_hash": kernel_source_hash(),
         }
         if world == 1 and not args.no_cpu_baseline:

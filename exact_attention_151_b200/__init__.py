@@ -16,7 +16,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
+__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
            "FA_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
 
@@ -32,7 +32,7 @@ FA_FP16 = 1
 
 # Every entry point declared in include/fa.h.
 EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen",
-                    "fa_status_sync", "fa_fwd_debug")
+                    "fa_fwd_splitkv", "fa_fwd_splitkv_plan", "fa_status_sync", "fa_fwd_debug")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -76,6 +76,12 @@ def load_library():
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32,
                                   i32, vp]
     lib.fa_fwd_varlen.restype = i32
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32, i32, vp,
+                                   ctypes.c_size_t, vp]
+    lib.fa_fwd_splitkv.restype = i32
+    lib.fa_fwd_splitkv_plan.argtypes = [i64, i64, i64, i64, i64, i32, ctypes.POINTER(i32),
+                                        ctypes.POINTER(ctypes.c_size_t)]
+    lib.fa_fwd_splitkv_plan.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
     _lib = lib
@@ -210,4 +216,49 @@ def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, scale: fl
                                           int(bool(causal)), _dtype_code(q), stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd_varlen")
+    return o, lse
+
+
+def splitkv_plan(B: int, Nq: int, Nk: int, Hq: int, D: int, num_splits: int = 0) -> tuple[int, int]:
+    """(number of key ranges, workspace bytes) fa_fwd_splitkv uses for these sizes on the current device."""
+    n = ctypes.c_int(0)
+    size = ctypes.c_size_t(0)
+    st = load_library().fa_fwd_splitkv_plan(B, Nq, Nk, Hq, D, int(num_splits), ctypes.byref(n), ctypes.byref(size))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv_plan")
+    return n.value, size.value
+
+
+def fwd_splitkv(q, k, v, scale: float | None = None, causal: bool = False, num_splits: int = 0, workspace=None,
+                o=None, lse=None):
+    """Split-KV forward (decode shapes): q [B,Nq,Hq,D], k/v [B,Nk,Hkv,D].
+
+    ``workspace`` is a CUDA uint8 tensor of at least splitkv_plan(...)[1] bytes
+    (allocated here with torch if omitted). Returns (o, lse) as fwd does.
+    """
+    import torch
+
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, _ = k.shape
+    _check_cuda(q=q, k=k, v=v)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    with torch.cuda.device(q.device):
+        _, need = splitkv_plan(B, Nq, Nk, Hq, D, num_splits)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+        _check_cuda(o=o, lse=lse)
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        st = load_library().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                           B, Nq, Nk, Hq, Hkv, D, ctypes.c_float(float(scale)), int(bool(causal)),
+                                           _dtype_code(q), int(num_splits), workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv")
     return o, lse

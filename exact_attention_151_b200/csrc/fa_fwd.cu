@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <mutex>
 
 #include "fa.h"
@@ -112,6 +113,10 @@ struct Shape {
   const int* cu_q;
   const int* cu_k;
   int64_t B, Nq, Nk, total_q, total_k, max_nq, Hq, Hkv, D;
+  int n_splits = 1;       // split-KV (dense shapes): number of key ranges
+  int split_tiles = 0;    // key tiles per range
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
 };
 
 template <int D, bool FP16>
@@ -171,7 +176,11 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.causal = causal ? 1 : 0;
   prm.wait_limit_ns = static_cast<unsigned long long>(limit_ns);
   prm.withhold_v_load = withhold;
-  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * sh.B * sh.Hq;
+  prm.n_splits = sh.n_splits;
+  prm.split_tiles = sh.split_tiles;
+  prm.part_o = sh.part_o;
+  prm.part_lse = sh.part_lse;
+  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * sh.B * sh.Hq * sh.n_splits;
   kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -179,15 +188,61 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (debug_enabled()) std::fprintf(stderr, "[fa] launch failed: %s\n", cudaGetErrorString(e));
     return FA_ERR_CUDA;
   }
+  if (sh.n_splits > 1) {
+    const int64_t rows = sh.B * sh.Hq * sh.Nq;
+    fa_splitkv_combine_kernel<D, FP16><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(
+        sh.part_o, sh.part_lse, static_cast<uint16_t*>(o), lse, sh.n_splits, static_cast<int>(sh.B * sh.Hq),
+        static_cast<int>(sh.Hq), static_cast<int>(sh.Nq));
+    const cudaError_t e2 = cudaGetLastError();
+    if (e2 != cudaSuccess) {
+      set_error("combine launch", e2);
+      return FA_ERR_CUDA;
+    }
+  }
   if (debug_enabled()) {
-    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d grid=%lld smem=%d\n",
+    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d splits=%d grid=%lld smem=%d\n",
                  D, FP16 ? "fp16" : "bf16", (long long)sh.B, (long long)sh.Nq, (long long)sh.Nk, (long long)sh.Hq,
-                 (long long)sh.Hkv, sh.cu_q ? "packed" : "dense", causal, (long long)grid, C::kSmemBytes);
+                 (long long)sh.Hkv, sh.cu_q ? "packed" : "dense", causal, sh.n_splits, (long long)grid, C::kSmemBytes);
   }
   return FA_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxSplits = 64;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of a split-KV call: fp32 partial O [n_splits, B*Hq, Nq, D], then
+// fp32 partial LSE [n_splits, B*Hq, Nq], each 256-byte aligned.
+size_t splitkv_bytes(int64_t n_splits, int64_t BH, int64_t Nq, int64_t D) {
+  return align256(static_cast<size_t>(n_splits * BH * Nq * D) * 4) + align256(static_cast<size_t>(n_splits * BH * Nq) * 4);
+}
+
+// Number of key ranges: when the query side alone fills less than half the
+// SMs, as many ranges as keep the CTAs within one wave (one CTA per SM), never
+// more than the key tiles or kMaxSplits; the count is then evened so every
+// range has the same number of tiles.
+int resolve_splits(int requested, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int sm_count, int* tiles_out) {
+  const int64_t n_kt = (Nk + kTile - 1) / kTile;
+  const int64_t base = ((Nq + kBlockRows - 1) / kBlockRows) * B * Hq;
+  int64_t want = requested;
+  if (want <= 0) want = (base >= sm_count / 2 || n_kt < 2) ? 1 : sm_count / base;
+  want = std::max<int64_t>(1, std::min<int64_t>({want, n_kt > 0 ? n_kt : 1, kMaxSplits}));
+  const int64_t tiles = (n_kt + want - 1) / want;
+  const int64_t splits = tiles > 0 ? (n_kt + tiles - 1) / tiles : 1;
+  *tiles_out = static_cast<int>(tiles);
+  return static_cast<int>(std::max<int64_t>(1, splits));
+}
+
+int device_sm_count(int dev) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& sh, float scale,
                    int causal, fa_dtype dtype, fa_stream_t stream, uint64_t limit_ns, int withhold) {
@@ -289,6 +344,57 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   try {
     if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
     fa::Shape sh{cu_seqlens_q, cu_seqlens_k, B, 0, 0, total_q, total_k, max_seqlen_q, Hq, Hkv, D};
+    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t D, int num_splits,
+                              int* splits_out, size_t* workspace_bytes) {
+  try {
+    if (!splits_out || !workspace_bytes || B < 0 || Nq < 0 || Nk < 0 || Hq < 0 || num_splits < 0)
+      return FA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      dev = -1;
+    }
+    const int sms = dev >= 0 ? fa::device_sm_count(dev) : 148;
+    int tiles = 0;
+    const int splits = fa::resolve_splits(num_splits, B, Nq, Nk, Hq, sms, &tiles);
+    *splits_out = splits;
+    *workspace_bytes = splits > 1 ? fa::splitkv_bytes(splits, B * Hq, Nq, D) : 0;
+    return FA_OK;
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t Nq,
+                         int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                         int num_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  try {
+    fa::Shape sh = fa::dense_shape(B, Nq, Nk, Hq, Hkv, D);
+    if (num_splits < 0) return FA_ERR_INVALID_ARG;
+    int splits = 1, tiles = 0;
+    size_t need = 0;
+    fa_status st = fa_fwd_splitkv_plan(B < 0 ? 0 : B, Nq < 0 ? 0 : Nq, Nk < 0 ? 0 : Nk, Hq < 0 ? 0 : Hq,
+                                       D, num_splits, &splits, &need);
+    if (st != FA_OK) return st;
+    if (splits > 1) {
+      if (!workspace || workspace_bytes < need) return FA_ERR_INVALID_ARG;
+      if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
+      int dev = 0;
+      cudaGetDevice(&dev);
+      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, fa::device_sm_count(dev), &tiles);
+      sh.n_splits = splits;
+      sh.split_tiles = tiles;
+      sh.part_o = static_cast<float*>(workspace);
+      sh.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             fa::align256(static_cast<size_t>(splits * B * Hq * Nq * D) * 4));
+    }
     return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
   } catch (...) {
     return FA_ERR_CUDA;

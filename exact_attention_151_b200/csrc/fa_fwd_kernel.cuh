@@ -252,6 +252,14 @@ struct Params {
   int n_blocks;         // ceil(max_nq / 256)
   float scale_log2;
   int causal;           // key j visible to query i iff j <= i + nk - nq (bottom-right aligned)
+  // Split-KV (n_splits > 1, dense shapes only): CTA split s covers key tiles
+  // [s * split_tiles, (s + 1) * split_tiles) and writes its own normalised O
+  // and LSE, in fp32, to part_o [n_splits, B, Hq, Nq, D] and part_lse
+  // [n_splits, B, Hq, Nq]; a separate kernel merges the splits.
+  int n_splits;
+  int split_tiles;
+  float* part_o;
+  float* part_lse;
   unsigned long long wait_limit_ns;
   int withhold_v_load;
 };
@@ -275,6 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
   const int causal = prm.causal;
 
+  // Split-KV index is the slowest-varying part of the block index.
+  const int split = static_cast<int>(blockIdx.x) / (prm.BH * prm.n_blocks);
+  const int xblk = static_cast<int>(blockIdx.x) - split * (prm.BH * prm.n_blocks);
   int bh, level;
   {
     // Causal: heads in groups of kHeadGroup; inside a group, query-block level
@@ -282,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // in L2 while its CTAs run, and the last CTAs to start are the lightest.
     const int per_group = kHeadGroup * prm.n_blocks;
     const int full_groups = prm.BH / kHeadGroup;
-    const int x = static_cast<int>(blockIdx.x);
+    const int x = xblk;
     int g, hg, within;
     if (x < full_groups * per_group) {
       g = x / per_group;
@@ -298,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (!causal) {
     // equal work per block: keep all blocks of a head adjacent (K/V shared in L2)
-    bh = static_cast<int>(blockIdx.x) / prm.n_blocks;
-    level = static_cast<int>(blockIdx.x) % prm.n_blocks;
+    bh = xblk / prm.n_blocks;
+    level = xblk % prm.n_blocks;
   }
   const int mb = causal ? (prm.n_blocks - 1 - level) : level;
   const int b = bh / prm.Hq;
@@ -339,8 +350,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (last_key < 0) return -1;
     return min(n_kt - 1, last_key / kTile);
   };
-  const int last0 = last_key_tile(qt0);
-  const int last1 = q1_valid ? last_key_tile(qt1) : -1;
+  // This CTA's key tiles: jb .. je-1 (all of them unless split-KV). Tile
+  // indices below are relative to jb; lastI is the last tile (relative) with a
+  // key visible to some row of query tile I, -1 if none.
+  const int jb = split * prm.split_tiles;
+  const int je = prm.n_splits > 1 ? min(n_kt, jb + prm.split_tiles) : n_kt;
+  auto last_rel = [&](int qt) -> int {
+    const int t = min(last_key_tile(qt), je - 1);
+    return t < jb ? -1 : t - jb;
+  };
+  const int last0 = last_rel(qt0);
+  const int last1 = q1_valid ? last_rel(qt1) : -1;
   const int n_kv = (last1 > last0 ? last1 : last0) + 1;
 
   if (threadIdx.x == 0) {
@@ -399,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, k0 + j * kTile, bar(C::kBarKFull + sk));
+          tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, k0 + (jb + j) * kTile, bar(C::kBarKFull + sk));
         nk = j + 1;
         const int sv = j % C::kVStages;
         if (j >= C::kVStages &&
@@ -408,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(withhold && j == 0)) {
           mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
           for (int hf = 0; hf < C::kHalves; ++hf)
-            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, k0 + j * kTile, bar(C::kBarVFull + sv));
+            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, k0 + (jb + j) * kTile, bar(C::kBarVFull + sv));
         }
         nv = j + 1;
       }
@@ -485,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv_half(i, j, sv, split, 1);
         return true;
       };
-      const bool split0 = split_p_tile(qt0, 0, causal, delta, nk);
-      const bool split1 = split_p_tile(qt1, 0, causal, delta, nk);
+      const bool split0 = jb == 0 && split_p_tile(qt0, 0, causal, delta, nk);
+      const bool split1 = jb == 0 && split_p_tile(qt1, 0, causal, delta, nk);
       bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
       for (int j = 0; ok && j <= n_kv; ++j) {
         const int sk = j % C::kKStages;
@@ -554,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kTile; ++k) s[k] = __uint_as_float(r[k / 32][k % 32]);
       }
-      const int kbase = j * kTile;
+      const int kbase = (jb + j) * kTile;
       if (kbase + kTile > nk || (causal && kbase + kTile - 1 > qt * kTile + delta)) {
         // last visible column of this row in this tile (may be < 0: none)
         const int lastcol = (causal ? min(nk - 1, qi + delta) : (nk - 1)) - kbase;
@@ -578,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(s * c - m) over the first 64 columns of S_i, published in two
       // halves (keys 0-63, 64-127) so the PV MMA can start on the first.
       float psum;
-      if (split_p_tile(qt, j, causal, delta, nk)) {
+      if (split_p_tile(qt, jb + j, causal, delta, nk)) {
         psum = softmax_exp_half<FP16, true, 0>(s, c, m_used, s_col);
       } else {
         psum = softmax_exp_half<FP16, false, 0>(s, c, m_used, s_col);
@@ -586,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + 2 * wg));
-      if (split_p_tile(qt, j, causal, delta, nk)) {
+      if (split_p_tile(qt, jb + j, causal, delta, nk)) {
         psum += softmax_exp_half<FP16, true, 1>(s, c, m_used, s_col);
       } else {
         psum += softmax_exp_half<FP16, false, 1>(s, c, m_used, s_col);
@@ -598,41 +618,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (last >= 0 && ok) ok = warp_wait_bar(bar(C::kBarOFinal + wg), 0, wc);
     // Epilogue. A row with no visible key (bottom-right causal with nq > nk,
-    // or nk == 0) gets O = 0 and LSE = -inf, whatever its TMEM lanes hold.
+    // or nk == 0; with split-KV: none in this split's key range) gets O = 0
+    // and LSE = -inf, whatever its TMEM lanes hold.
+    const bool splitkv = prm.n_splits > 1;
+    const int row_last_key = causal ? min(nk - 1, qi + delta) : nk - 1;
     const bool row_valid = (wg == 0 || q1_valid) && qi < nq;
-    const bool row_has_keys = nk > 0 && (!causal || qi + delta >= 0);
-    uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + h) * D;
-    float* lse_at = prm.lse + (prm.cu_q != nullptr
-                                   ? static_cast<int64_t>(h) * prm.total_q + q0 + qi
-                                   : (static_cast<int64_t>(b) * prm.Hq + h) * prm.Nq + qi);
-    if (last >= 0 && ok) {
-      tc_fence_after();
-      const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
+    const bool row_has_keys = row_last_key >= 0 && (!splitkv || row_last_key >= jb * kTile);
+    if (splitkv) {
+      // fp32 partial result of this key range (normalised by its own sum)
+      const int64_t prow = (static_cast<int64_t>(split) * prm.BH + bh) * prm.Nq + qi;
+      float* orow = prm.part_o + prow * D;
+      if (last >= 0 && ok) {
+        tc_fence_after();
+        const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t o[32];
-        tmem_ld32(o_col + q * 32, o);
-        tmem_wait_ld();
-        uint32_t pk[16];
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(o_col + q * 32, o);
+          tmem_wait_ld();
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float2 v = fmul2(make_float2(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1])),
-                                 make_float2(inv_l, inv_l));
-          pk[k] = row_has_keys ? pack2<FP16>(v.x, v.y) : 0u;
+            for (int k = 0; k < 8; ++k) {
+              const float2 a = fmul2(make_float2(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1])),
+                                     make_float2(inv_l, inv_l));
+              const float2 c2 = fmul2(make_float2(__uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3])),
+                                      make_float2(inv_l, inv_l));
+              dst[k] = row_has_keys ? make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(c2.x),
+                                                 __float_as_uint(c2.y))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
         }
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+        if (row_valid) prm.part_lse[prow] = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+      } else if (last < 0 && row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-        }
+        for (int k = 0; k < D / 4; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+        prm.part_lse[prow] = -INFINITY;
       }
-      if (row_valid) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
-    } else if (last < 0 && row_valid) {
-      // no key tile at all for this query tile
-      uint4* dst = reinterpret_cast<uint4*>(orow);
+    } else {
+      uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + h) * D;
+      float* lse_at = prm.lse + (prm.cu_q != nullptr
+                                     ? static_cast<int64_t>(h) * prm.total_q + q0 + qi
+                                     : (static_cast<int64_t>(b) * prm.Hq + h) * prm.Nq + qi);
+      if (last >= 0 && ok) {
+        tc_fence_after();
+        const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
 #pragma unroll
-      for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
-      *lse_at = -INFINITY;
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(o_col + q * 32, o);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float2 v = fmul2(make_float2(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1])),
+                                   make_float2(inv_l, inv_l));
+            pk[k] = row_has_keys ? pack2<FP16>(v.x, v.y) : 0u;
+          }
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
+        }
+        if (row_valid) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+      } else if (last < 0 && row_valid) {
+        // no key tile at all for this query tile
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+        *lse_at = -INFINITY;
+      }
     }
   }
 
@@ -642,6 +700,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Split-KV merge: for every (b, h, i), with the splits' partial results
+// (O_s normalised by its own sum, LSE_s = log of that sum):
+//   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s,
+// the same online-softmax rescaling as inside the kernel, applied once across
+// splits (empty splits have LSE_s = -inf and weight 0; if every split is empty
+// O = 0 and LSE = -inf). One warp per query row; D / 32 columns per lane.
+template <int D, bool FP16>
+__global__ void __launch_bounds__(128) fa_splitkv_combine_kernel(const float* __restrict__ part_o,
+                                                                 const float* __restrict__ part_lse,
+                                                                 uint16_t* __restrict__ out, float* __restrict__ lse,
+                                                                 int n_splits, int BH, int Hq, int Nq) {
+  const int lane = threadIdx.x % 32;
+  const int64_t rowid = static_cast<int64_t>(blockIdx.x) * 4 + threadIdx.x / 32;  // (bh, i)
+  const int64_t rows = static_cast<int64_t>(BH) * Nq;
+  if (rowid >= rows) return;
+  const int64_t stride = rows;  // between splits
+  float mx = -INFINITY;
+  for (int sp = lane; sp < n_splits; sp += 32) mx = fmaxf(mx, part_lse[sp * stride + rowid]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  const int bh = static_cast<int>(rowid / Nq), i = static_cast<int>(rowid % Nq);
+  const int b = bh / Hq, h = bh % Hq;
+  uint16_t* orow = out + ((static_cast<int64_t>(b) * Nq + i) * Hq + h) * D;
+  constexpr int kPer = D / 32;  // columns per lane
+  if (mx == -INFINITY) {
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) orow[lane * kPer + c] = 0;
+    if (lane == 0) lse[rowid] = -INFINITY;
+    return;
+  }
+  float acc[kPer];
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+  float wsum = 0.f;
+  for (int sp = 0; sp < n_splits; ++sp) {
+    const float w = ex2_approx((part_lse[sp * stride + rowid] - mx) * 1.44269504088896340736f);
+    wsum += w;
+    const float* src = part_o + (sp * stride + rowid) * D + lane * kPer;
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] = fmaf(w, src[c], acc[c]);
+  }
+  const float inv = 1.f / wsum;
+#pragma unroll
+  for (int c = 0; c < kPer; c += 2) {
+    const uint32_t pk = pack2<FP16>(acc[c] * inv, acc[c + 1] * inv);
+    *reinterpret_cast<uint32_t*>(orow + lane * kPer + c) = pk;
+  }
+  if (lane == 0) lse[rowid] = mx + lg2_approx(wsum) * kLn2;
 }
 
 }  // namespace fa

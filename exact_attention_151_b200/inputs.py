@@ -36,6 +36,9 @@ class Workload:
     v_dist: str = "normal"  # "normal" (N(0,1)) or "uniform" (U(-1, 1))
     seed: int = 0
     scale: float | None = None  # None means 1/sqrt(D)
+    Nk: int | None = None  # key length (None: N); queries are N long
+    Hkv: int | None = None  # key/value heads (None: H)
+    splitkv: bool = False  # run through the split-KV entry point
     notes: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -43,15 +46,33 @@ class Workload:
         return self.scale if self.scale is not None else 1.0 / math.sqrt(self.D)
 
     @property
+    def n_keys(self) -> int:
+        return self.N if self.Nk is None else self.Nk
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.Hkv is None else self.Hkv
+
+    @property
     def flops(self) -> float:
-        """4*B*H*N^2*D, halved when causal (the metric's counting convention)."""
-        f = 4.0 * self.B * self.H * self.N * self.N * self.D
-        return f / 2 if self.causal else f
+        """4*D flops per visible (query, key) pair: 4*B*H*N^2*D, halved when
+        causal (the metric's counting convention) for square problems; the
+        exact visible-pair count (bottom-right causal mask) otherwise."""
+        nq, nk = self.N, self.n_keys
+        if nq == nk:
+            f = 4.0 * self.B * self.H * nq * nq * self.D
+            return f / 2 if self.causal else f
+        if self.causal:
+            pairs = sum(min(nk, max(0, i + nk - nq + 1)) for i in range(nq))
+        else:
+            pairs = nq * nk
+        return 4.0 * self.B * self.H * pairs * self.D
 
     @property
     def min_hbm_bytes(self) -> int:
         """Read Q, K, V once, write O once (16-bit) and LSE (fp32)."""
-        return 8 * self.B * self.N * self.H * self.D + 4 * self.B * self.H * self.N
+        q_side = 4 * self.B * self.N * self.H * self.D + 4 * self.B * self.H * self.N
+        return q_side + 4 * self.B * self.n_keys * self.kv_heads * self.D
 
     def with_(self, **kw) -> "Workload":
         d = dict(self.__dict__)
@@ -79,20 +100,27 @@ WORKLOADS: dict[str, Workload] = {
         # stated regime); the configuration as written peaks near 25-30.
         Workload("stress_hot_b2h16n4093d64_fp16_causal", B=2, N=4093, H=16, D=64, dtype="fp16", causal=True,
                  q_std=16.0, v_dist="uniform"),
+        # Split-KV (decoding): one query per head against a long key sequence,
+        # grouped-query heads (32 query heads over 8 K/V heads).
+        Workload("decode_b1h32kv8nq1nk32768d128_splitkv", B=1, N=1, Nk=32768, H=32, Hkv=8, D=128, causal=True,
+                 splitkv=True),
+        Workload("decode_b8h32kv8nq1nk8192d128_splitkv", B=8, N=1, Nk=8192, H=32, Hkv=8, D=128, causal=True,
+                 splitkv=True),
     ]
 }
 
 
 def make_qkv(w: Workload, seed: int | None = None):
-    """Return (q, k, v) as contiguous CPU tensors of w.dtype in [B, N, H, D]."""
+    """Return (q [B, N, H, D], k and v [B, Nk, Hkv, D]) as contiguous CPU tensors of w.dtype."""
     g = torch.Generator().manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.N, w.H, w.D)
+    kshape = (w.B, w.n_keys, w.kv_heads, w.D)
     q = torch.randn(shape, generator=g, dtype=torch.float32) * w.q_std
-    k = torch.randn(shape, generator=g, dtype=torch.float32) * w.k_std
+    k = torch.randn(kshape, generator=g, dtype=torch.float32) * w.k_std
     if w.v_dist == "uniform":
-        v = torch.rand(shape, generator=g, dtype=torch.float32) * 2.0 - 1.0
+        v = torch.rand(kshape, generator=g, dtype=torch.float32) * 2.0 - 1.0
     else:
-        v = torch.randn(shape, generator=g, dtype=torch.float32)
+        v = torch.randn(kshape, generator=g, dtype=torch.float32)
     dt = TORCH_DTYPES[w.dtype]
     return q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous()
 

@@ -35,6 +35,7 @@
 #ifndef FA_B200_FA_H_
 #define FA_B200_FA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -131,6 +132,33 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
                         const int32_t* cu_seqlens_k, int64_t B, int64_t max_seqlen_q, int64_t total_q, int64_t total_k,
                         int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
                         fa_stream_t stream);
+
+/*
+ * fa_fwd_splitkv - fa_fwd_gqa with the keys cut into ranges processed by
+ * separate CTAs, for shapes whose query side alone cannot fill the GPU
+ * (decoding: few queries per head, long key sequences). Each range writes its
+ * partial O (normalised by its own sum, fp32) and LSE to `workspace`; a
+ * second kernel merges them with weights exp(LSE_r - LSE). Same arguments,
+ * layouts, masks and errors as fa_fwd_gqa, plus:
+ *   num_splits       : 0 = choose (enough CTAs for every SM), else requested
+ *                      count; capped at 64 and at the number of 128-key tiles
+ *   workspace        : device memory, 256-byte aligned, owned by the caller,
+ *                      at least the size fa_fwd_splitkv_plan reports; unused
+ *                      (may be NULL) when the plan has one range
+ *   workspace_bytes  : its size; too small -> FA_ERR_INVALID_ARG, no launch
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t Nq,
+                         int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
+                         int num_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_fwd_splitkv_plan - number of key ranges fa_fwd_splitkv will use for
+ * these sizes on the current device, and the workspace it needs in bytes
+ * (0 when it uses one range). Host only; launches nothing.
+ */
+fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t D, int num_splits,
+                              int* splits_out, size_t* workspace_bytes);
 
 /*
  * fa_status_sync - synchronise `stream`, then read and clear this device's
