@@ -32,7 +32,8 @@ FA_FP16 = 1
 
 # Every entry point declared in include/fa.h.
 EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen",
-                    "fa_fwd_splitkv", "fa_fwd_splitkv_plan", "fa_status_sync", "fa_fwd_debug")
+                    "fa_fwd_splitkv", "fa_fwd_splitkv_plan", "fa_fwd_splitkv_noalloc", "fa_status_sync",
+                    "fa_fwd_debug")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -82,6 +83,9 @@ def load_library():
     lib.fa_fwd_splitkv_plan.argtypes = [i64, i64, i64, i64, i64, i32, ctypes.POINTER(i32),
                                         ctypes.POINTER(ctypes.c_size_t)]
     lib.fa_fwd_splitkv_plan.restype = i32
+    lib.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32,
+                                           i32, vp]
+    lib.fa_fwd_splitkv_noalloc.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
     _lib = lib
@@ -262,3 +266,29 @@ def fwd_splitkv(q, k, v, scale: float | None = None, causal: bool = False, num_s
     if st != FA_OK:
         raise FaError(st, "fa_fwd_splitkv")
     return o, lse
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def fwd_splitkv_noalloc(q, k, v, o, lse, scale: float | None = None, causal: bool = False, num_splits: int = 0):
+    """Split-KV forward whose partial results use the library's built-in scratch
+    buffer instead of a caller workspace, so the call allocates no device memory
+    (for callers that cannot allocate on the call path). ``o`` and ``lse`` are
+    caller-provided as in fwd_into. Calls overlapping on the GPU share the
+    scratch and race; sizes needing more than NOALLOC_SCRATCH_BYTES of partial
+    results raise FaError(FA_ERR_UNSUPPORTED)."""
+    import torch
+
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, _ = k.shape
+    _check_cuda(q=q, k=k, v=v, o=o, lse=lse)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = load_library().fa_fwd_splitkv_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                                   lse.data_ptr(), B, Nq, Nk, Hq, Hkv, D, ctypes.c_float(float(scale)),
+                                                   int(bool(causal)), _dtype_code(q), int(num_splits), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv_noalloc")

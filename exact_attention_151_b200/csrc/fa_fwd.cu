@@ -300,6 +300,39 @@ Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, in
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- no-allocation scratch
+// Scratch for fa_fwd_splitkv_noalloc: a fixed-size buffer compiled into the
+// library, so that entry point needs no device allocation at all. Every GPU
+// that loads the library holds it (kNoAllocScratchBytes) until the process
+// exits. In host code `g_noalloc_scratch` only names the symbol; its device
+// address is looked up per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of the scratch on the current device `dev`, looked up once per
+// device (cudaGetSymbolAddress; no allocation) and cached.
+fa_status noalloc_scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      set_error("cudaGetSymbolAddress(scratch)", e);
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return FA_OK;
+}
+
 }  // namespace fa
 
 extern "C" {
@@ -393,6 +426,48 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
       sh.split_tiles = tiles;
       sh.part_o = static_cast<float*>(workspace);
       sh.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             fa::align256(static_cast<size_t>(splits * B * Hq * Nq * D) * 4));
+    }
+    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                                 int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal,
+                                 fa_dtype dtype, int num_splits, fa_stream_t stream) {
+  try {
+    if (num_splits < 0 || B < 0 || Nq < 0 || Nk < 0 || Hq < 0) return FA_ERR_INVALID_ARG;
+    int splits = 1;
+    size_t need = 0;
+    fa_status st = fa_fwd_splitkv_plan(B, Nq, Nk, Hq, D, num_splits, &splits, &need);
+    if (st != FA_OK) return st;
+    if (need > fa::kNoAllocScratchBytes) {
+      std::snprintf(fa::g_last_error, sizeof(fa::g_last_error),
+                    "split-KV scratch of %zu bytes needed, the built-in scratch holds %zu bytes", need,
+                    fa::kNoAllocScratchBytes);
+      return FA_ERR_UNSUPPORTED;
+    }
+    fa::Shape sh = fa::dense_shape(B, Nq, Nk, Hq, Hkv, D);
+    if (splits > 1) {
+      int dev = 0;
+      const cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) {
+        fa::set_error("cudaGetDevice", e);
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      if (dev < 0 || dev >= fa::kMaxDevices) return FA_ERR_UNSUPPORTED;
+      void* scratch = nullptr;
+      st = fa::noalloc_scratch_address(dev, &scratch);
+      if (st != FA_OK) return st;
+      int tiles = 0;
+      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, fa::device_sm_count(dev), &tiles);
+      sh.n_splits = splits;
+      sh.split_tiles = tiles;
+      sh.part_o = static_cast<float*>(scratch);
+      sh.part_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) +
                                              fa::align256(static_cast<size_t>(splits * B * Hq * Nq * D) * 4));
     }
     return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);

@@ -161,6 +161,36 @@ fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int
                               int* splits_out, size_t* workspace_bytes);
 
 /*
+ * fa_fwd_splitkv_noalloc - fa_fwd_splitkv without a workspace argument, for
+ * callers that must not allocate device memory on the call path: for example
+ * a serving loop whose GPU memory is reserved up front by another allocator,
+ * or code that cannot handle an out-of-memory failure in the middle of a
+ * request. The pages describe no such entry point; it has no counterpart
+ * there.
+ *
+ *   Arguments, layouts, masks and results as fa_fwd_splitkv; the caller still
+ *   provides q, k, v, o and lse.
+ *   The partial results go to a scratch buffer compiled into the library:
+ *   FA_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every GPU which
+ *   loads the library holds until the process exits. Sizes whose partial
+ *   results would not fit (fa_fwd_splitkv_plan's workspace_bytes above that)
+ *   return FA_ERR_UNSUPPORTED without launching, with the sizes in
+ *   fa_last_error().
+ *   No cudaMalloc, cudaFree or other allocating call is made. The first call
+ *   on each device looks up the scratch buffer's device address
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture on that device.
+ *   Every call uses the same buffer and leaves its last contents there;
+ *   nothing in it has to start at zero (each call overwrites every entry it
+ *   reads). Calls that overlap on the GPU (different streams, or the same
+ *   buffer used concurrently) race with each other and give wrong results.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                                 int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal,
+                                 fa_dtype dtype, int num_splits, fa_stream_t stream);
+
+/*
  * fa_status_sync - synchronise `stream`, then read and clear this device's
  * status word. Returns FA_OK; FA_ERR_TIMEOUT if a kernel on this device gave
  * up on a bounded wait since the last call (its outputs are then invalid);
