@@ -63,6 +63,9 @@ def _load():
         lib.oracle_attention_varlen.argtypes = [u16p, u16p, u16p, i64p, i64p, i64, i64, i64, i64, ctypes.c_double,
                                                 ctypes.c_int, ctypes.c_int, f64p, f64p, ctypes.c_int]
         lib.oracle_attention_varlen.restype = ctypes.c_int
+        lib.oracle_attention_backward.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_double,
+                                                  ctypes.c_int, ctypes.c_int, f64p, f64p, f64p, ctypes.c_int]
+        lib.oracle_attention_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -163,6 +166,25 @@ def attention_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool, dtype: str
     if rc:
         raise ValueError(f"oracle_attention_varlen failed ({rc})")
     return o, lse
+
+
+def attention_backward(q, k, v, dout, scale: float, causal: bool, dtype: str, nthreads: int | None = None):
+    """Gradients (dQ, dK, dV), float64 [B, N, H, D], of sum(O * dO) through the
+    definition; all inputs are 16-bit patterns in [B, N, H, D]."""
+    q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
+    B, N, H, D = _shape(q, k, v)
+    if dout.shape != q.shape:
+        raise ValueError("dO must match q")
+    dq = np.empty((B, N, H, D), dtype=np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    rc = _load().oracle_attention_backward(
+        _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16), _ptr(dout, ctypes.c_uint16),
+        B, N, H, D, float(scale), int(bool(causal)), DTYPE_CODES[dtype], _ptr(dq, ctypes.c_double),
+        _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), int(nthreads or default_threads()))
+    if rc:
+        raise ValueError(f"oracle_attention_backward failed ({rc})")
+    return dq, dk, dv
 
 
 def tiled_reference(q, k, v, scale: float, causal: bool, dtype: str, block_size: int = 128):

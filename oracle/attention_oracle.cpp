@@ -284,6 +284,83 @@ int oracle_attention_varlen(const uint16_t* q, const uint16_t* k, const uint16_t
   return 0;
 }
 
+// Backward of the definition: the gradients of a scalar loss L through O,
+// given dO = dL/dO (the recomputation-based backward the jsqmd page describes
+// needs exactly these quantities; the weights are recomputed from Q, K and the
+// row's log-sum-exp rather than stored). For each (b, h), with
+// P_ij = exp(s_ij - LSE_i) over the visible j (0 elsewhere):
+//   dV_j  = sum_i P_ij dO_i
+//   dP_ij = dO_i . V_j
+//   D_i   = dO_i . O_i              (= sum_j P_ij dP_ij)
+//   dS_ij = P_ij (dP_ij - D_i)
+//   dQ_i  = scale * sum_j dS_ij K_j
+//   dK_j  = scale * sum_i dS_ij Q_i
+// O and LSE are the fp64 forward of this file. Inputs are 16-bit patterns in
+// [B, N, H, D] (dO too); gradients are double in [B, N, H, D].
+int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                              int64_t B, int64_t N, int64_t H, int64_t D, double scale, int causal, int dtype,
+                              double* dq, double* dk, double* dv, int nthreads) {
+  Problem p{q, k, v, B, N, H, D, scale, causal, dtype};
+  if (!valid(p) || !dout || !dq || !dk || !dv) return 1;
+  std::vector<double> Q, K, V, dO;
+  std::vector<double> P(static_cast<size_t>(N) * static_cast<size_t>(N));
+  std::vector<double> dS(static_cast<size_t>(N) * static_cast<size_t>(N));
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t h = 0; h < H; ++h) {
+      widen_head(p, q, b, h, Q);
+      widen_head(p, k, b, h, K);
+      widen_head(p, v, b, h, V);
+      widen_head(p, dout, b, h, dO);
+      // rows: P, O, D, dP, dS
+      parallel_for(N, nthreads, [&](int64_t lo, int64_t hi) {
+        std::vector<double> s(static_cast<size_t>(N)), orow(static_cast<size_t>(D));
+        for (int64_t i = lo; i < hi; ++i) {
+          const int64_t nvis = visible_count(p, i);
+          score_row(p, Q, K, i, nvis, s.data());
+          const double lse = finish_row(p, s.data(), nvis, V, orow.data());
+          double Di = 0.0;
+          for (int64_t d = 0; d < D; ++d) Di += dO[i * D + d] * orow[d];
+          for (int64_t j = 0; j < N; ++j) {
+            if (j < nvis) {
+              const double pij = std::exp(s[j] - lse);
+              double dpij = 0.0;
+              for (int64_t d = 0; d < D; ++d) dpij += dO[i * D + d] * V[j * D + d];
+              P[i * N + j] = pij;
+              dS[i * N + j] = pij * (dpij - Di);
+            } else {
+              P[i * N + j] = 0.0;
+              dS[i * N + j] = 0.0;
+            }
+          }
+        }
+      });
+      // dQ rows
+      parallel_for(N, nthreads, [&](int64_t lo, int64_t hi) {
+        for (int64_t i = lo; i < hi; ++i)
+          for (int64_t d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < N; ++j) acc += dS[i * N + j] * K[j * D + d];
+            dq[at(p, b, i, h, d)] = scale * acc;
+          }
+      });
+      // dK, dV rows
+      parallel_for(N, nthreads, [&](int64_t lo, int64_t hi) {
+        for (int64_t j = lo; j < hi; ++j)
+          for (int64_t d = 0; d < D; ++d) {
+            double ak = 0.0, av = 0.0;
+            for (int64_t i = 0; i < N; ++i) {
+              ak += dS[i * N + j] * Q[i * D + d];
+              av += P[i * N + j] * dO[i * D + d];
+            }
+            dk[at(p, b, j, h, d)] = scale * ak;
+            dv[at(p, b, j, h, d)] = av;
+          }
+      });
+    }
+  }
+  return 0;
+}
+
 // The handbook's tiled online-softmax routine, in fp64, one (b, h) at a time.
 // For every query block [qs, qe) and every key block [ks, ke) (both cut at
 // block_size, the last one truncated at N):
