@@ -1,4 +1,4 @@
-"""B200-native exact attention forward: O = softmax(scale * Q K^T [+ causal]) V and per-row LSE.
+"""B200-native exact attention: O = softmax(scale * Q K^T [+ causal]) V with per-row LSE, and its gradients.
 
 Thin Python binding over the C ABI in ``include/fa.h`` (library
 ``libfa_b200.so``, built in-tree for sm_100a). This module only marshals
@@ -16,7 +16,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "status_sync", "FaError", "library_path", "load_library",
+__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "bwd", "bwd_workspace_size", "status_sync", "FaError", "library_path", "load_library",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
            "FA_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
 
@@ -33,7 +33,7 @@ FA_FP16 = 1
 # Every entry point declared in include/fa.h.
 EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen",
                     "fa_fwd_splitkv", "fa_fwd_splitkv_plan", "fa_fwd_splitkv_noalloc", "fa_status_sync",
-                    "fa_fwd_debug")
+                    "fa_fwd_debug", "fa_bwd", "fa_bwd_workspace_size")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -86,6 +86,11 @@ def load_library():
     lib.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32,
                                            i32, vp]
     lib.fa_fwd_splitkv_noalloc.restype = i32
+    lib.fa_bwd_workspace_size.argtypes = [i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.fa_bwd_workspace_size.restype = i32
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, i32, i32, vp,
+                           ctypes.c_size_t, vp]
+    lib.fa_bwd.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
     _lib = lib
@@ -292,3 +297,54 @@ def fwd_splitkv_noalloc(q, k, v, o, lse, scale: float | None = None, causal: boo
                                                    int(bool(causal)), _dtype_code(q), int(num_splits), stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd_splitkv_noalloc")
+
+
+def bwd_workspace_size(B: int, N: int, H: int) -> int:
+    """Device workspace bytes fa_bwd needs for these sizes."""
+    size = ctypes.c_size_t(0)
+    st = load_library().fa_bwd_workspace_size(int(B), int(N), int(H), ctypes.byref(size))
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd_workspace_size")
+    return size.value
+
+
+def bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False, dq=None, dk=None, dv=None,
+        workspace=None):
+    """Gradients (dq, dk, dv) of sum(O * dout) for the forward's q, k, v [B,N,H,D], o and lse.
+
+    ``o`` and ``lse`` are what fwd returned for the same q, k, v, scale and
+    causal. dq/dk/dv (like q) and ``workspace`` (CUDA uint8, at least
+    bwd_workspace_size(B, N, H) bytes) are allocated here if omitted.
+    """
+    import torch
+
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("q, k, v, o and dout must all be [B, N, H, D]")
+    B, N, H, D = q.shape
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    for t in (k, v, o, dout):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, o and dout must share one dtype")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for t in (dq, dk, dv):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("dq, dk and dv must be like q")
+    with torch.cuda.device(q.device):
+        need = bwd_workspace_size(B, N, H)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        _check_cuda(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace)
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D,
+                                   ctypes.c_float(float(scale)), int(bool(causal)), code, workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv

@@ -21,7 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "fa_fwd.cu")]
-HEADERS = [os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "fa_fwd_kernel.cuh"), os.path.join(INCLUDE, "fa.h")]
+HEADERS = [os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "fa_fwd_kernel.cuh"), os.path.join(CSRC, "fa_bwd_kernel.cuh"),
+           os.path.join(INCLUDE, "fa.h")]
 
 
 def nvcc_path() -> str:

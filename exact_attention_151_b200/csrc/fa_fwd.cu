@@ -1,6 +1,7 @@
-// fa_fwd.cu - host side of the fused exact-attention forward: argument
-// checks, TMA tensor-map encoding, launch, and the C ABI declared in fa.h.
-// The kernel itself is in fa_fwd_kernel.cuh.
+// fa_fwd.cu - host side of the fused exact attention: argument checks, TMA
+// tensor-map encoding, launches, and the C ABI declared in fa.h. The forward
+// kernel is in fa_fwd_kernel.cuh, the backward kernels in fa_bwd_kernel.cuh
+// (one translation unit, so every kernel reports into one status word).
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -15,6 +16,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -299,6 +301,126 @@ Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, in
   return sh;
 }
 
+// ---------------------------------------------------------------- backward
+
+// Workspace of the backward: D_i = dO_i . O_i, then LSE_i log2(e), each fp32
+// [B*H, Npad] with Npad = N rounded up to whole 128-row tiles, 256-byte aligned.
+size_t bwd_ws_bytes(int64_t B, int64_t N, int64_t H) {
+  const int64_t npad = (N + kTile - 1) / kTile * kTile;
+  return 2 * align256(static_cast<size_t>(B * H * npad) * 4);
+}
+
+template <int D, bool FP16, bool KV_SIDE>
+fa_status bwd_launch(int dev, const CUtensorMap& x1, const CUtensorMap& x2, const CUtensorMap& y1,
+                     const CUtensorMap& y2, const bwd::Params& prm, int64_t grid, cudaStream_t stream) {
+  using C = bwd::Cfg<D>;
+  auto kernel = bwd::fa_bwd_kernel<D, FP16, KV_SIDE>;
+  const unsigned bit = 1u << (4 + (D == 128 ? 4 : 0) + (FP16 ? 2 : 0) + (KV_SIDE ? 1 : 0));
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!(g_devices[dev].configured & bit)) {
+      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+      if (e != cudaSuccess) {
+        set_error("cudaFuncSetAttribute(backward)", e);
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      g_devices[dev].configured |= bit;
+    }
+  }
+  kernel<<<static_cast<unsigned>(grid), bwd::kThreads, C::kSmemBytes, stream>>>(x1, x2, y1, y2, prm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error(KV_SIDE ? "backward dK/dV launch" : "backward dQ launch", e);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+template <int D, bool FP16>
+fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, float scale,
+                  int causal, void* workspace, cudaStream_t stream) {
+  const int64_t n_tiles = (N + kTile - 1) / kTile;
+  const int64_t npad = n_tiles * kTile;
+  const int64_t BH = B * H;
+  float* ws_d = static_cast<float*>(workspace);
+  float* ws_l = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BH * npad) * 4));
+  const int64_t prep_blocks = (BH * npad + 7) / 8;
+  bwd::fa_bwd_prep_kernel<D, FP16><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(BH),
+      static_cast<int>(N), static_cast<int>(H), static_cast<int>(npad));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("backward preprocess launch", e);
+    return FA_ERR_CUDA;
+  }
+  const bool fp16 = FP16;
+  CUtensorMap tq, tk, tv, tdo;
+  if (make_tmap(&tq, q, B * N, H, D, fp16) != FA_OK || make_tmap(&tk, k, B * N, H, D, fp16) != FA_OK ||
+      make_tmap(&tv, v, B * N, H, D, fp16) != FA_OK || make_tmap(&tdo, dout, B * N, H, D, fp16) != FA_OK)
+    return FA_ERR_CUDA;
+  bwd::Params prm;
+  prm.ws_d = ws_d;
+  prm.ws_l = ws_l;
+  prm.N = static_cast<int>(N);
+  prm.H = static_cast<int>(H);
+  prm.Npad = static_cast<int>(npad);
+  prm.n_tiles = static_cast<int>(n_tiles);
+  // same base-2 factor as the forward (see launch)
+  float c = scale * 1.44269504088896340736f;
+  if (std::fabs(c) < FLT_MIN) c = std::signbit(c) ? -FLT_MIN : FLT_MIN;
+  prm.scale_log2 = c;
+  prm.scale = scale;
+  prm.causal = causal ? 1 : 0;
+  prm.wait_limit_ns = kDefaultWaitLimitNs;
+  const int64_t grid = n_tiles * BH;
+  prm.out0 = static_cast<uint16_t*>(dq);
+  prm.out1 = nullptr;
+  fa_status st = bwd_launch<D, FP16, false>(dev, tq, tdo, tk, tv, prm, grid, stream);
+  if (st != FA_OK) return st;
+  prm.out0 = static_cast<uint16_t*>(dk);
+  prm.out1 = static_cast<uint16_t*>(dv);
+  st = bwd_launch<D, FP16, true>(dev, tk, tv, tq, tdo, prm, grid, stream);
+  if (st != FA_OK) return st;
+  if (debug_enabled())
+    std::fprintf(stderr, "[fa] bwd D=%d %s B=%lld N=%lld H=%lld causal=%d grid=2x%lld\n", D, FP16 ? "fp16" : "bf16",
+                 (long long)B, (long long)N, (long long)H, causal, (long long)grid);
+  return FA_OK;
+}
+
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
+                   fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (B < 0 || N < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (B * N > INT32_MAX - 2 * kTile || H > INT32_MAX || B * H > INT32_MAX / ((N + kTile - 1) / kTile + 1))
+    return FA_ERR_UNSUPPORTED;
+  if (static_cast<double>(B) * N * H * D * 2 >= 1099511627776.0) return FA_ERR_UNSUPPORTED;
+  if (B * H * ((N + kTile - 1) / kTile * kTile) / 8 >= INT32_MAX) return FA_ERR_UNSUPPORTED;  // preprocess grid
+  if (workspace_bytes < bwd_ws_bytes(B, N, H)) return FA_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv), static_cast<const void*>(lse)})
+    if (!aligned16(p)) return FA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
+  int dev = 0;
+  fa_status st = check_device(&dev);
+  if (st != FA_OK) return st;
+  st = load_encoder();
+  if (st != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool fp16 = dtype == FA_FP16;
+  if (D == 128)
+    return fp16 ? bwd_run<128, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s)
+                : bwd_run<128, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s);
+  return fp16 ? bwd_run<64, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s)
+              : bwd_run<64, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- no-allocation scratch
@@ -482,6 +604,23 @@ fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, flo
   try {
     return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream,
                         wait_limit_ns, withhold_v_load ? 1 : 0);
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspace_bytes) {
+  if (!workspace_bytes || B < 0 || N < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  *workspace_bytes = fa::bwd_ws_bytes(B, N, H);
+  return FA_OK;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
+                 fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  try {
+    return fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H, D, scale, causal, dtype, workspace,
+                        workspace_bytes, stream);
   } catch (...) {
     return FA_ERR_CUDA;
   }

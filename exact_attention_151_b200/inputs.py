@@ -125,6 +125,14 @@ def make_qkv(w: Workload, seed: int | None = None):
     return q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous()
 
 
+def make_dout(w: Workload, seed: int | None = None):
+    """Output gradient dO [B, N, H, D] for the backward: N(0, 1) from its own
+    generator (seed + 7919, a stated choice), rounded to w.dtype."""
+    g = torch.Generator().manual_seed((w.seed if seed is None else seed) + 7919)
+    d = torch.randn((w.B, w.N, w.H, w.D), generator=g, dtype=torch.float32)
+    return d.to(TORCH_DTYPES[w.dtype]).contiguous()
+
+
 def bits(t: torch.Tensor):
     """Raw 16-bit patterns of a CPU bf16/fp16 tensor as a numpy uint16 array."""
     import numpy as np

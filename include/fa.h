@@ -1,5 +1,5 @@
 /*
- * fa.h - C ABI of the B200 (sm_100a) fused exact-attention forward.
+ * fa.h - C ABI of the B200 (sm_100a) fused exact attention (forward and backward).
  *
  * The operation (one call):
  *   O[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) * v[b,j,h,:]
@@ -198,6 +198,49 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
  * FA_ERR_CUDA if the synchronisation itself failed.
  */
 fa_status fa_status_sync(fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size - bytes of device workspace fa_bwd needs for these
+ * sizes: two fp32 arrays [B*H, ceil(N/128)*128], each rounded up to 256 bytes.
+ * Returns FA_ERR_INVALID_ARG for a NULL output or a negative size.
+ */
+fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspace_bytes);
+
+/*
+ * fa_bwd - gradients of the forward above, enqueued on `stream`.
+ *
+ * Given dO = dL/dO, with P[i,j] = exp(scale q_i.k_j - LSE_i) over the
+ * visible keys (the forward's weights, recomputed from q, k and lse rather
+ * than stored: jsqmd.com "Flash Attention applications", core-mechanism
+ * section, item 3 "Recomputation"), D_i = dO_i . O_i and
+ * dS[i,j] = P[i,j] (dO_i . v_j - D_i):
+ *   dV_j = sum_i P[i,j] dO_i,  dQ_i = scale sum_j dS[i,j] k_j,
+ *   dK_j = scale sum_i dS[i,j] q_i        (per batch and head).
+ * The result is deterministic: no atomics, every output element is written
+ * by exactly one thread, with a fixed summation order (the deterministic
+ * mode of mlqm.cn FA1/FA2 comparison, section 3.2).
+ *
+ *   q, k, v, o, dout : device, [B, N, H, D], dtype `dtype` (read only); o and
+ *                      lse are the forward's outputs for these q, k, v, scale
+ *                      and causal
+ *   lse              : device, float32 [B, H, N] (read only)
+ *   dq, dk, dv       : device, [B, N, H, D], dtype `dtype` (written; must not
+ *                      overlap the inputs)
+ *   D                : 64 or 128;  scale, causal, dtype : as in fa_fwd
+ *   workspace        : device, at least fa_bwd_workspace_size(B, N, H) bytes,
+ *                      256-byte aligned; owned by the caller, scratch for the
+ *                      duration of the call (stream-ordered)
+ * Three kernels run in stream order: D and LSE log2(e) into the workspace,
+ * then dQ (one CTA per 128-query tile), then dK and dV (one CTA per 128-key
+ * tile). fp32 accumulation in Tensor Memory; P and dS enter the tensor cores
+ * rounded to `dtype`.
+ * Errors: as fa_fwd; additionally FA_ERR_INVALID_ARG for a NULL or too small
+ * workspace and FA_ERR_MISALIGNED for a workspace not 256-byte aligned.
+ * B, N or H == 0 returns FA_OK without launching.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
+                 fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_fwd_debug - fa_fwd with two test hooks (same arguments first).

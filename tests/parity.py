@@ -52,3 +52,40 @@ def sample_rows(B: int, H: int, N: int, per_head_random: int, seed: int = 0, hea
         rows.update(rng.integers(0, N, size=per_head_random).tolist())
         out.extend((b, h, i) for i in sorted(rows))
     return np.array(out, dtype=np.int64)
+
+
+# Backward (dQ, dK, dV). Each gradient element is a sum of products whose
+# 16-bit factor (P or dS, rounded once before the tensor cores) carries a
+# relative error up to u (bf16 2^-8, fp16 2^-11), and the result is rounded to
+# the same dtype once more: with independent roundings the expected relative
+# L2 error is about 0.8 u (3.2e-3 bf16, 4e-4 fp16); the bound allows about 3x
+# (bf16) and 4x (fp16) that. The error of one element is about 0.8 u times its
+# own scale (the root of the sum of its squared terms), so the largest error
+# is compared with the largest reference magnitude: a 5-sigma error on the
+# largest-scale elements is about 4 u of that scale, and the bound is 5 u.
+# (Relative to the RMS instead, causal gradients would be penalised for the
+# spread of their magnitudes: early keys collect terms from many queries.)
+TOL_GRAD_REL_L2 = {"bf16": 1e-2, "fp16": 2e-3}
+TOL_GRAD_MAX_REL = {"bf16": 5 * 2.0**-8, "fp16": 5 * 2.0**-11}
+
+
+def grad_metrics(got, ref) -> dict:
+    out = {}
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        g = np.asarray(g, dtype=np.float64)
+        r = np.asarray(r, dtype=np.float64)
+        diff = g - r
+        rn = float(np.linalg.norm(r))
+        rmax = float(np.abs(r).max(initial=0.0))
+        dmax = float(np.abs(diff).max(initial=0.0))
+        out[name] = {
+            "rel_l2": float(np.linalg.norm(diff) / rn) if rn > 0 else float(np.linalg.norm(diff)),
+            "max_rel": dmax / rmax if rmax > 0 else dmax,
+            "finite": bool(np.isfinite(g).all()),
+        }
+    return out
+
+
+def grad_passes(m: dict, dtype: str) -> bool:
+    return all(x["finite"] and x["rel_l2"] <= TOL_GRAD_REL_L2[dtype] and x["max_rel"] <= TOL_GRAD_MAX_REL[dtype]
+               for x in m.values())

@@ -79,3 +79,35 @@ def test_general_entry_points_validate_before_any_device_call():
     # varlen head dim not supported
     assert lib.fa_fwd_varlen(P, P, P, P, P, P, P, 2, 16, 32, 32, 4, 4, 96, f32(0.1), 0, fa.FA_BF16, 0) == \
         fa.FA_ERR_UNSUPPORTED
+
+
+def _bwd(lib, q=P, o=P, lse=P, dq=P, ws=P, B=1, N=16, H=1, D=64, scale=0.125, dtype=fa.FA_BF16, ws_bytes=1 << 20):
+    f32 = __import__("ctypes").c_float
+    return lib.fa_bwd(q, P, P, o, lse, P, dq, P, P, B, N, H, D, f32(scale), 0, dtype, ws, ws_bytes, 0)
+
+
+def test_backward_validates_before_any_device_call():
+    lib = fa.load_library()
+    assert _bwd(lib, q=0) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, dq=0) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, ws=0) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, ws_bytes=16) == fa.FA_ERR_INVALID_ARG            # workspace too small
+    assert _bwd(lib, B=-1) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, dtype=9) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(lib, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert _bwd(lib, o=P + 8) == fa.FA_ERR_MISALIGNED
+    assert _bwd(lib, ws=P + 16) == fa.FA_ERR_MISALIGNED                # workspace must be 256-byte aligned
+    assert _bwd(lib, q=0, o=0, lse=0, dq=0, ws=0, N=0) == fa.FA_OK    # empty: no-op
+
+
+def test_backward_workspace_size():
+    # two fp32 arrays [B*H, N rounded up to 128], each rounded up to 256 bytes
+    assert fa.bwd_workspace_size(2, 300, 3) == 2 * (2 * 3 * 384 * 4)
+    assert fa.bwd_workspace_size(1, 1, 1) == 2 * 512
+    assert fa.bwd_workspace_size(0, 5, 5) == 0
+    lib = fa.load_library()
+    import ctypes
+    size = ctypes.c_size_t(0)
+    assert lib.fa_bwd_workspace_size(-1, 5, 5, ctypes.byref(size)) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_workspace_size(1, 5, 5, None) == fa.FA_ERR_INVALID_ARG
