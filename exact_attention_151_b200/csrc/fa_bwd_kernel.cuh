@@ -11,17 +11,30 @@
 //                        whole 128-row tiles (pad rows: D = 0, LSE = +inf, so
 //                        their weights are exactly 0);
 //   fa_bwd_kernel<.., KV_SIDE = false>  one CTA per (128-query tile, b, h):
-//                        S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - D)
-//                        by one thread per query row, dQ += dS K;
+//                        S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - D),
+//                        dQ += dS K over the key tiles;
 //   fa_bwd_kernel<.., KV_SIDE = true>   one CTA per (128-key tile, b, h):
-//                        S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T
-//                        by one thread per key row, dV += P^T dO, dK += dS^T Q.
-// Both share one warp-specialised skeleton: a TMA loader warp (the tile's two
-// fixed operands once, the streamed pair into a two-stage ring), an MMA warp
-// (converged, one elected lane issues tcgen05.mma), and four compute warps
-// (TMEM lane = row). The operand of the accumulating MMAs that comes from the
-// elementwise step (dS, P^T, dS^T) is written back to TMEM as 16-bit pairs
-// over the first half of the score's columns, as P is in the forward.
+//                        S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and
+//                        dS^T, dV += P^T dO and dK += dS^T Q over the query
+//                        tiles.
+//
+// One warp-specialised skeleton serves both: a TMA loader warp (the tile's
+// two fixed operands once, the streamed pair into a two-stage ring), an MMA
+// warp (converged, one elected lane issues tcgen05.mma) and two compute
+// warpgroups that split each 128-column score tile into halves (TMEM lane =
+// row, warpgroup h = columns 64h .. 64h+63). A compute thread keeps its 64
+// weights P in registers between its two phases: A reads S and forms P,
+// B reads dP and forms dS. The 16-bit MMA operands they produce go back to
+// TMEM inside the half's own columns.
+//
+// The MMA warp interleaves consecutive streamed tiles so that the tensor
+// cores work while the warpgroups compute:
+//   key side:   S(0) dP(0) | dV(t) S(t+1) dK(t) dP(t+1) | ...
+//   query side: S(0) dP(0) | S(t+1) dQ(t) dP(t+1) | ...
+// Each accumulating product is issued per half, as soon as that half's
+// operand is in TMEM. Score products keep N = 128: the tensor cores read both
+// operands of a shared-memory product from shared memory, and at N = 64 that
+// read, not the math, sets the pace.
 #pragma once
 
 #include <cuda.h>
@@ -33,9 +46,10 @@
 namespace fa {
 namespace bwd {
 
-constexpr int kThreads = 192;
-constexpr int kMma = 4;   // warp index
-constexpr int kLoad = 5;  // warp index
+constexpr int kThreads = 320;  // warps 0-7: compute warpgroups 0 and 1, 8: MMA, 9: loader
+constexpr int kMma = 8;        // warp index
+constexpr int kLoad = 9;       // warp index
+constexpr int kGroup = 16;     // heads per scheduling group (causal)
 
 template <int D>
 struct Cfg {
@@ -49,18 +63,23 @@ struct Cfg {
   static constexpr int kBarX = 0;
   static constexpr int kBarYFull = 1;                 // [kStages]
   static constexpr int kBarYEmpty = 1 + kStages;      // [kStages]
-  static constexpr int kBarSFull = 1 + 2 * kStages;   // scores ready
-  static constexpr int kBarPFull = kBarSFull + 1;     // elementwise results written (128 arrivals)
-  static constexpr int kBarDone = kBarPFull + 1;      // last accumulating MMA finished
+  static constexpr int kBarSFull = 1 + 2 * kStages;   // scores S (or S^T) in TMEM
+  static constexpr int kBarDPFull = kBarSFull + 1;    // dP (or dP^T) in TMEM
+  static constexpr int kBarA = kBarDPFull + 1;        // [2] phase A of warpgroup h done (128 arrivals)
+  static constexpr int kBarB = kBarA + 2;             // [2] phase B of warpgroup h done (128 arrivals)
+  static constexpr int kBarDone = kBarB + 2;          // last accumulating MMA finished
   static constexpr int kBarDrain = kBarDone + 1;
   static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kWsOff = kBarOff + 128;    // per compute warp 2 x 128 floats (key side)
-  static constexpr int kMiscOff = kWsOff + 4 * 1024;
+  static constexpr int kWsOff = kBarOff + 128;        // key side: per compute warp -LSE log2(e), -D of 64 queries
+  static constexpr int kMiscOff = kWsOff + 8 * 512;
   static_assert(kNumBars * 8 <= 128, "barrier area");
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  // TMEM columns: score A (S or S^T), score B (dP or dP^T), accumulators
-  static constexpr uint32_t kColSA = 0, kColSB = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+  // TMEM columns: scores (S or S^T), dP (or dP^T), accumulators. Key side:
+  // acc0 = dK, acc1 = dV. Query side: acc0 = dQ, and dS (16-bit pairs, 32
+  // columns per half) at acc1.
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+  static_assert(256 + 2 * D <= 512, "TMEM budget");
 };
 
 struct Params {
@@ -68,7 +87,7 @@ struct Params {
   const float* ws_l;    // [B*H, Npad]: LSE_i * log2(e) (+inf on pad rows)
   uint16_t* out0;       // query side: dQ;   key side: dK
   uint16_t* out1;       // key side: dV
-  int N, H, Npad, n_tiles;
+  int N, H, BH, Npad, n_tiles;
   float scale_log2;     // scale * log2(e)
   float scale;
   int causal;
@@ -110,6 +129,95 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
   }
 }
 
+// Phase A for one thread's half row: p = 2^(s c + nl) for the 64 scores of
+// TMEM columns kColS + 64h .. (two 32-column chunks). nl is -LSE log2(e):
+// per row (query side, `nl_row`) or per column from shared memory (key side,
+// `nl_col`). MASKED tiles (the causal diagonal or the ragged tail) zero the
+// invisible entries through the exponent and use the MUFU exp only; other
+// tiles send every fourth pair through the FMA-pipe polynomial. With PACK the
+// 16-bit weights are stored to the half's first 32 columns (key side: P^T).
+template <bool FP16, bool KV_SIDE, bool MASKED, bool PACK>
+__device__ __forceinline__ void phase_a(uint32_t t_s, float c, float nl_row, const float* nl_col, int first_col,
+                                        int row_abs, int n_valid, int causal, float (&p)[64]) {
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t sa[32];
+    tmem_ld32(t_s + ch * 32, sa);
+    tmem_wait_ld();
+    uint32_t pk[16];
+    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = ch * 32 + 2 * q;  // element index in the half
+      float2 nl;
+      if constexpr (KV_SIDE) {  // 16-byte broadcast reads (the buffer is 16-byte aligned)
+        if ((q & 1) == 0) v4 = *reinterpret_cast<const float4*>(nl_col + e);
+        nl = (q & 1) ? make_float2(v4.z, v4.w) : make_float2(v4.x, v4.y);
+      } else {
+        nl = make_float2(nl_row, nl_row);
+      }
+      float2 x = ffma2(make_float2(__uint_as_float(sa[2 * q]), __uint_as_float(sa[2 * q + 1])), c2, nl);
+      float2 pp;
+      if constexpr (MASKED) {
+        const int c0 = first_col + e;  // column index (query on the key side, key on the query side)
+        bool v0, v1;
+        if constexpr (KV_SIDE) {  // row = key row_abs; pad queries already carry -inf through nl
+          v0 = !causal || c0 >= row_abs;
+          v1 = !causal || c0 + 1 >= row_abs;
+        } else {                  // row = query row_abs
+          v0 = c0 < n_valid && (!causal || c0 <= row_abs);
+          v1 = c0 + 1 < n_valid && (!causal || c0 + 1 <= row_abs);
+        }
+        x.x = v0 ? x.x : -INFINITY;
+        x.y = v1 ? x.y : -INFINITY;
+        pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      } else {
+        if (emulated_pair(ch * 16 + q)) {
+          pp = exp2_poly2(x);
+        } else {
+          pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        }
+      }
+      p[e] = pp.x;
+      p[e + 1] = pp.y;
+      if constexpr (PACK) pk[q] = pack2<FP16>(pp.x, pp.y);
+    }
+    if constexpr (PACK) tmem_st16(t_s + ch * 16, pk);
+  }
+}
+
+// Phase B for one thread's half row: ds = p (dp + nd) for the 64 dP values of
+// TMEM columns t_dp .. (two chunks), nd = -D per row (query side) or per column
+// (key side); the 16-bit dS pairs go to t_out .. t_out + 31.
+template <bool FP16, bool KV_SIDE>
+__device__ __forceinline__ void phase_b(uint32_t t_dp, uint32_t t_out, float nd_row, const float* nd_col,
+                                        const float (&p)[64]) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t sb[32];
+    tmem_ld32(t_dp + ch * 32, sb);
+    tmem_wait_ld();
+    uint32_t pk[16];
+    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = ch * 32 + 2 * q;
+      float2 nd;
+      if constexpr (KV_SIDE) {
+        if ((q & 1) == 0) v4 = *reinterpret_cast<const float4*>(nd_col + e);
+        nd = (q & 1) ? make_float2(v4.z, v4.w) : make_float2(v4.x, v4.y);
+      } else {
+        nd = make_float2(nd_row, nd_row);
+      }
+      const float2 g = fadd2(make_float2(__uint_as_float(sb[2 * q]), __uint_as_float(sb[2 * q + 1])), nd);
+      const float2 ds = fmul2(make_float2(p[e], p[e + 1]), g);
+      pk[q] = pack2<FP16>(ds.x, ds.y);
+    }
+    tmem_st16(t_out + ch * 16, pk);
+  }
+}
+
 // KV_SIDE = false: tile of 128 queries; X1 = Q, X2 = dO fixed, stream (K_t, V_t)
 //   over key tiles t = 0 .. last; out0 = dQ.
 // KV_SIDE = true:  tile of 128 keys; X1 = K, X2 = V fixed, stream (Q_t, dO_t)
@@ -133,8 +241,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
   const int N = prm.N;
   const int causal = prm.causal;
-  const int tile = static_cast<int>(blockIdx.x) % prm.n_tiles;  // this CTA's query (or key) tile
-  const int bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
+  // CTA -> (bh, tile). Causal work per tile is uneven (query tile i streams
+  // i + 1 key tiles; key tile j streams n_tiles - j query tiles): CTAs go in
+  // groups of kGroup heads, heaviest tiles first within a group, so the last
+  // wave holds the short ones and a group's K/V (or Q/dO) stay L2-resident.
+  // Non-causal: head-major.
+  int tile, bh;
+  if (causal) {
+    const int per_group = kGroup * prm.n_tiles;
+    const int g = static_cast<int>(blockIdx.x) / per_group;
+    const int r = static_cast<int>(blockIdx.x) % per_group;
+    const int gsize = min(kGroup, prm.BH - g * kGroup);
+    const int level = r / gsize;
+    bh = g * kGroup + r % gsize;
+    tile = KV_SIDE ? level : prm.n_tiles - 1 - level;
+  } else {
+    tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
+    bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
+  }
   const int b = bh / prm.H, h = bh % prm.H;
   // streamed tiles: query side: keys 0 .. (causal ? tile : n_tiles-1);
   //                 key side:   queries (causal ? tile : 0) .. n_tiles-1
@@ -149,7 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarYEmpty + s), 1);
     }
     mbar_init(bar(C::kBarSFull), 1);
-    mbar_init(bar(C::kBarPFull), 128);
+    mbar_init(bar(C::kBarDPFull), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::kBarA + i), 128);
+      mbar_init(bar(C::kBarB + i), 128);
+    }
     mbar_init(bar(C::kBarDone), 1);
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
@@ -208,152 +336,183 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t x_desc0 = smem_desc_sw128(x_smem(0), 16, 1024);  // K-major views
     const uint64_t y_desc0 = smem_desc_sw128(y_smem(0, 0), 16, 1024);
     const uint64_t y_mn0 = smem_desc_sw128(y_smem(0, 0), C::kSlabBytes, 1024);  // MN-major view of the same tiles
-    bool ok = warp_wait_bar(bar(C::kBarX), 0, wc);
+    // score product into TMEM column `col`: X_i Y_i(stage s)^T, K = D in steps of 16
+    auto issue_score = [&](int i, int s, uint32_t col) {
+      const uint64_t a = x_desc0 + static_cast<uint64_t>(i) * kTileStep;
+      const uint64_t bb = y_desc0 + static_cast<uint64_t>(2 * s + i) * kTileStep;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
+        mma_ss_elect(tmem + col, a + off, bb + off, idesc_score, kk > 0 ? 1u : 0u);
+      }
+    };
+    // accumulating product for half hf of the streamed tile's 128 rows:
+    // acc += A(TMEM, 16-bit pairs from a_col) * Y_i(stage s) rows 64hf .. (MN-major B)
+    auto issue_acc = [&](uint32_t acc_col, uint32_t a_col, int i, int s, int hf, bool first) {
+      const uint64_t bb = y_mn0 + static_cast<uint64_t>(2 * s + i) * kTileStep;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = 4 * hf + q;
+        mma_ts_elect(tmem + acc_col, tmem + a_col + q * 8, bb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_acc,
+                     (first && q == 0) ? 0u : 1u);
+      }
+    };
+    bool ok = warp_wait_bar(bar(C::kBarX), 0, wc) && warp_wait_bar(bar(C::kBarYFull), 0, wc);
+    if (ok) {
+      tc_fence_after();
+      issue_score(0, 0, C::kColS);
+      mma_commit_elect(bar(C::kBarSFull));
+      issue_score(1, 0, C::kColDP);
+      mma_commit_elect(bar(C::kBarDPFull));
+    }
     for (int t = 0; ok && t < n_t; ++t) {
       const int s = t % C::kStages;
-      ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
-      if (!ok) break;
-      tc_fence_after();
-      // score A = X1 Y1^T (S or S^T), score B = X2 Y2^T (dP or dP^T); K = D in steps of 16
-      const uint64_t y1 = y_desc0 + static_cast<uint64_t>(2 * s) * kTileStep;
-      const uint64_t y2 = y1 + kTileStep;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
-        mma_ss_elect(tmem + C::kColSA, x_desc0 + off, y1 + off, idesc_score, kk > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
-        mma_ss_elect(tmem + C::kColSB, x_desc0 + kTileStep + off, y2 + off, idesc_score, kk > 0 ? 1u : 0u);
-      }
-      mma_commit_elect(bar(C::kBarSFull));
-      ok = warp_wait_bar(bar(C::kBarPFull), static_cast<uint32_t>(t & 1), wc);
-      if (!ok) break;
-      tc_fence_after();
-      // accumulate: K = 128 rows of the streamed tiles in steps of 16 (B operand MN-major)
-      const uint64_t y1mn = y_mn0 + static_cast<uint64_t>(2 * s) * kTileStep;
-      const uint64_t y2mn = y1mn + kTileStep;
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-        const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-        if constexpr (KV_SIDE) {
-          mma_ts_elect(tmem + C::kColAcc1, tmem + C::kColSA + kk * 8, y2mn + off, idesc_acc, acc);  // dV += P^T dO
-          mma_ts_elect(tmem + C::kColAcc0, tmem + C::kColSB + kk * 8, y1mn + off, idesc_acc, acc);  // dK += dS^T Q
-        } else {
-          mma_ts_elect(tmem + C::kColAcc0, tmem + C::kColSA + kk * 8, y1mn + off, idesc_acc, acc);  // dQ += dS K
+      const bool more = t + 1 < n_t;
+      const uint32_t ph = static_cast<uint32_t>(t & 1);
+      const uint32_t ph_next = static_cast<uint32_t>(((t + 1) / C::kStages) & 1);
+      if constexpr (KV_SIDE) {
+        // dV += P^T dO per half as each warpgroup publishes its P^T
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
+          if (ok) {
+            tc_fence_after();
+            issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, s, hf, t == 0 && hf == 0);
+          }
         }
+        if (!ok) break;
+        // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
+        if (more) {
+          ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_score(0, (t + 1) % C::kStages, C::kColS);
+          mma_commit_elect(bar(C::kBarSFull));
+        }
+        // dK += dS^T Q per half
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
+          if (ok) {
+            tc_fence_after();
+            issue_acc(C::kColAcc0, C::kColDP + 64 * hf, 0, s, hf, t == 0 && hf == 0);
+          }
+        }
+        if (!ok) break;
+      } else {
+        // both warpgroups have read S: the next tile's S may overwrite it
+        ok = warp_wait_bar(bar(C::kBarA), ph, wc) && warp_wait_bar(bar(C::kBarA + 1), ph, wc);
+        if (!ok) break;
+        if (more) {
+          ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_score(0, (t + 1) % C::kStages, C::kColS);
+          mma_commit_elect(bar(C::kBarSFull));
+        }
+        // dQ += dS K per half
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
+          if (ok) {
+            tc_fence_after();
+            issue_acc(C::kColAcc0, C::kColAcc1 + 32 * hf, 0, s, hf, t == 0 && hf == 0);
+          }
+        }
+        if (!ok) break;
       }
       if (t + C::kStages < n_t) mma_commit_elect(bar(C::kBarYEmpty + s));
-      if (t == n_t - 1) mma_commit_elect(bar(C::kBarDone));
+      if (more) {
+        // dP of the next tile (after the accumulating products that read this tile's dS)
+        issue_score(1, (t + 1) % C::kStages, C::kColDP);
+        mma_commit_elect(bar(C::kBarDPFull));
+      } else {
+        mma_commit_elect(bar(C::kBarDone));
+      }
     }
     if (!ok) {
       mma_commit_elect(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0);
     }
   } else {
-    // ------------------------------------------------------------ compute warps (TMEM lane = row)
-    const int row = warp * 32 + lane;
-    const int r_abs = tile * kTile + row;  // this thread's query (or key) index
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
+    const int wg = warp / 4;                  // column half of every score tile
+    const int qd = warp % 4;                  // TMEM lane quadrant
+    const int row = qd * 32 + lane;
+    const int r_abs = tile * kTile + row;     // this thread's query (or key) index
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const float c = prm.scale_log2;
     const float* ws_d = prm.ws_d + static_cast<int64_t>(bh) * prm.Npad;
     const float* ws_l = prm.ws_l + static_cast<int64_t>(bh) * prm.Npad;
-    float row_d = 0.f, row_l = 0.f;
+    float nl_row = 0.f, nd_row = 0.f;
     if constexpr (!KV_SIDE) {
-      row_d = ws_d[r_abs];
-      row_l = ws_l[r_abs];
+      nl_row = -ws_l[r_abs];
+      nd_row = -ws_d[r_abs];
     }
-    // key side: each warp keeps its own copy of the current query tile's
-    // LSE log2(e) and D values (warp-local, so no barrier across warps)
-    float* ws_s_l = reinterpret_cast<float*>(smem + C::kWsOff) + warp * 2 * kTile;
-    float* ws_s_d = ws_s_l + kTile;
+    // key side: this warp's copy of -LSE log2(e) and -D for its 64 query columns
+    float* nl_col = reinterpret_cast<float*>(smem + C::kWsOff) + warp * 128;
+    float* nd_col = nl_col + 64;
+    const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
+    const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
+    const uint32_t t_ds = KV_SIDE ? t_dp : tmem + lane_base + C::kColAcc1 + 32 * wg;
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
-      const int cbase = (t_first + t) * kTile;  // first column index (key, or query) of this tile
+      const int cbase = (t_first + t) * kTile;  // first column (key, or query) of this tile
+      const int first_col = cbase + 64 * wg;
+      const uint32_t ph = static_cast<uint32_t>(t & 1);
       if constexpr (KV_SIDE) {
         __syncwarp();  // every lane is done with the previous tile's values
 #pragma unroll
-        for (int i = 0; i < kTile / 32; ++i) {
-          ws_s_l[i * 32 + lane] = ws_l[cbase + i * 32 + lane];
-          ws_s_d[i * 32 + lane] = ws_d[cbase + i * 32 + lane];
+        for (int i = 0; i < 2; ++i) {
+          nl_col[i * 32 + lane] = -ws_l[first_col + i * 32 + lane];
+          nd_col[i * 32 + lane] = -ws_d[first_col + i * 32 + lane];
         }
         __syncwarp();
       }
-      ok = warp_wait_bar(bar(C::kBarSFull), static_cast<uint32_t>(t & 1), wc);
+      const bool masked = (causal && cbase == tile * kTile) || cbase + kTile > N;
+      ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
       if (!ok) break;
       tc_fence_after();
-      // Columns in chunks of 32: the 16-bit results of chunk ch go to packed
-      // columns 16 ch .. 16 ch + 15, which only hold scores already read.
-      const bool masked = KV_SIDE ? (causal && cbase == tile * kTile)
-                                  : (cbase + kTile > N || (causal && cbase == tile * kTile));
-#pragma unroll
-      for (int ch = 0; ch < kTile / 32; ++ch) {
-        uint32_t sa[32], sb[32];
-        tmem_ld32(tmem + lane_base + C::kColSA + ch * 32, sa);
-        tmem_ld32(tmem + lane_base + C::kColSB + ch * 32, sb);
-        tmem_wait_ld();
-        uint32_t pk_a[16], pk_b[16];  // query side: dS (pk_a); key side: P^T (pk_a), dS^T (pk_b)
-#pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          float p[2], ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float sv = __uint_as_float(sa[q + e]);
-            const float dpv = __uint_as_float(sb[q + e]);
-            const int cidx = cbase + ch * 32 + q + e;
-            if constexpr (KV_SIDE) {
-              // row = key r_abs, column = query cidx; pad queries have LSE = +inf, so P = 0
-              const bool vis = !masked || cidx >= r_abs;
-              p[e] = vis ? ex2_approx(fmaf(sv, c, -ws_s_l[ch * 32 + q + e])) : 0.f;
-              ds[e] = p[e] * (dpv - ws_s_d[ch * 32 + q + e]);
-            } else {
-              // row = query r_abs, column = key cidx
-              const bool vis = !masked || (cidx < N && (!causal || cidx <= r_abs));
-              p[e] = vis ? ex2_approx(fmaf(sv, c, -row_l)) : 0.f;
-              ds[e] = p[e] * (dpv - row_d);
-            }
-          }
-          if constexpr (KV_SIDE) {
-            pk_a[q / 2] = pack2<FP16>(p[0], p[1]);
-            pk_b[q / 2] = pack2<FP16>(ds[0], ds[1]);
-          } else {
-            pk_a[q / 2] = pack2<FP16>(ds[0], ds[1]);
-          }
-        }
-        tmem_st16(tmem + lane_base + C::kColSA + ch * 16, pk_a);
-        if constexpr (KV_SIDE) tmem_st16(tmem + lane_base + C::kColSB + ch * 16, pk_b);
+      float p[64];
+      if (masked) {
+        phase_a<FP16, KV_SIDE, true, KV_SIDE>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
+      } else {
+        phase_a<FP16, KV_SIDE, false, KV_SIDE>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
       }
+      if constexpr (KV_SIDE) tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarA + wg));
+      ok = warp_wait_bar(bar(C::kBarDPFull), ph, wc);
+      if (!ok) break;
+      tc_fence_after();
+      phase_b<FP16, KV_SIDE>(t_dp, t_ds, nd_row, nd_col, p);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull));
+      mbar_arrive(bar(C::kBarB + wg));
     }
     if (ok) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
     if (ok) {
       tc_fence_after();
+      // key side: warpgroup 0 writes dK (scaled), warpgroup 1 dV; query side:
+      // warpgroup h writes dQ columns h D/2 .. (scaled)
       const bool row_valid = r_abs < N;
-      const int64_t obase = ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
+      uint16_t* dst_row = (KV_SIDE && wg == 1 ? prm.out1 : prm.out0) +
+                          ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
+      const float mul = (KV_SIDE && wg == 1) ? 1.f : prm.scale;
+      constexpr int kCols = KV_SIDE ? D : D / 2;
+      const uint32_t acc = tmem + lane_base + (KV_SIDE ? (wg == 0 ? C::kColAcc0 : C::kColAcc1)
+                                                       : C::kColAcc0 + wg * (D / 2));
+      const int col0 = KV_SIDE ? 0 : wg * (D / 2);
 #pragma unroll
-      for (int which = 0; which < (KV_SIDE ? 2 : 1); ++which) {
-        // query side: dQ (scaled); key side: which 0 = dK (scaled, acc0), 1 = dV (acc1)
-        const uint32_t col = which == 0 ? C::kColAcc0 : C::kColAcc1;
-        const float mul = which == 0 ? prm.scale : 1.f;
-        uint16_t* dst_row = (which == 0 ? prm.out0 : prm.out1) + obase;
+      for (int q = 0; q < kCols / 32; ++q) {
+        uint32_t a[32];
+        tmem_ld32(acc + q * 32, a);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t a[32];
-          tmem_ld32(tmem + lane_base + col + q * 32, a);
-          tmem_wait_ld();
-          uint32_t pk[16];
+        for (int k = 0; k < 16; ++k)
+          pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + col0 + q * 32);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul);
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-          }
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
     }

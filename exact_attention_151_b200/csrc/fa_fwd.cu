@@ -365,6 +365,7 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
   prm.ws_l = ws_l;
   prm.N = static_cast<int>(N);
   prm.H = static_cast<int>(H);
+  prm.BH = static_cast<int>(BH);
   prm.Npad = static_cast<int>(npad);
   prm.n_tiles = static_cast<int>(n_tiles);
   // same base-2 factor as the forward (see launch)
