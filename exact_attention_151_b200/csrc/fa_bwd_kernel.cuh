@@ -94,38 +94,53 @@ struct Params {
   unsigned long long wait_limit_ns;
 };
 
-// D_i and LSE_i log2(e) per row, padded to whole tiles. One warp per row.
+// D_i and LSE_i log2(e) per row into the tile-padded workspace. Blocks below
+// n_real_blocks read O and dO in memory order ([B, N, H, D] rows, D / 8
+// threads per row, 16-byte loads); the rest fill the pad rows (D = 0,
+// LSE = +inf).
 template <int D, bool FP16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __restrict__ o,
                                                           const uint16_t* __restrict__ dout,
                                                           const float* __restrict__ lse, float* __restrict__ ws_d,
-                                                          float* __restrict__ ws_l, int BH, int N, int H, int Npad) {
-  const int lane = threadIdx.x % 32;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x / 32;  // (bh, i) over the padded rows
-  if (r >= static_cast<int64_t>(BH) * Npad) return;
-  const int bh = static_cast<int>(r / Npad), i = static_cast<int>(r % Npad);
-  if (i >= N) {
-    if (lane == 0) {
-      ws_d[r] = 0.f;
-      ws_l[r] = INFINITY;
+                                                          float* __restrict__ ws_l, int B, int N, int H, int Npad,
+                                                          unsigned n_real_blocks) {
+  constexpr int kLanes = D / 8;                 // threads per row
+  constexpr int kRowsPerBlock = 256 / kLanes;
+  const int64_t n_rows = static_cast<int64_t>(B) * N * H;
+  if (blockIdx.x < n_real_blocks) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanes;  // (b N + i) H + h
+    const int sub = threadIdx.x % kLanes;
+    const bool valid = row < n_rows;
+    float acc = 0.f;
+    if (valid) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
+      const uint4 y = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 a = unpack2<FP16>(xs[k]);
+        const float2 c = unpack2<FP16>(ys[k]);
+        acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+      }
     }
-    return;
-  }
-  const int b = bh / H, h = bh % H;
-  const int64_t base = ((static_cast<int64_t>(b) * N + i) * H + h) * D;
-  constexpr int kPer = D / 32;  // elements per lane (2 or 4)
-  float acc = 0.f;
 #pragma unroll
-  for (int c = 0; c < kPer; c += 2) {
-    const float2 x = unpack2<FP16>(*reinterpret_cast<const uint32_t*>(o + base + lane * kPer + c));
-    const float2 y = unpack2<FP16>(*reinterpret_cast<const uint32_t*>(dout + base + lane * kPer + c));
-    acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    ws_d[r] = acc;
-    ws_l[r] = lse[static_cast<int64_t>(bh) * N + i] * 1.44269504088896340736f;
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid && sub == 0) {
+      const int h = static_cast<int>(row % H);
+      const int64_t bi = row / H;
+      const int i = static_cast<int>(bi % N);
+      const int64_t bh = (bi / N) * H + h;
+      ws_d[bh * Npad + i] = acc;
+      ws_l[bh * Npad + i] = lse[bh * N + i] * 1.44269504088896340736f;
+    }
+  } else {
+    const int pad = Npad - N;
+    const int64_t p = static_cast<int64_t>(blockIdx.x - n_real_blocks) * 256 + threadIdx.x;
+    if (pad > 0 && p < static_cast<int64_t>(B) * H * pad) {
+      const int64_t idx = (p / pad) * Npad + N + p % pad;
+      ws_d[idx] = 0.f;
+      ws_l[idx] = INFINITY;
+    }
   }
 }
 

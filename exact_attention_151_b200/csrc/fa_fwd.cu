@@ -346,10 +346,12 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
   const int64_t BH = B * H;
   float* ws_d = static_cast<float*>(workspace);
   float* ws_l = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BH * npad) * 4));
-  const int64_t prep_blocks = (BH * npad + 7) / 8;
-  bwd::fa_bwd_prep_kernel<D, FP16><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
-      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(BH),
-      static_cast<int>(N), static_cast<int>(H), static_cast<int>(npad));
+  constexpr int64_t kPrepRows = 256 / (D / 8);  // rows per preprocess block
+  const int64_t real_blocks = (B * N * H + kPrepRows - 1) / kPrepRows;
+  const int64_t pad_blocks = (BH * (npad - N) + 255) / 256;
+  bwd::fa_bwd_prep_kernel<D, FP16><<<static_cast<unsigned>(real_blocks + pad_blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(B),
+      static_cast<int>(N), static_cast<int>(H), static_cast<int>(npad), static_cast<unsigned>(real_blocks));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("backward preprocess launch", e);
@@ -402,7 +404,8 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   if (B * N > INT32_MAX - 2 * kTile || H > INT32_MAX || B * H > INT32_MAX / ((N + kTile - 1) / kTile + 1))
     return FA_ERR_UNSUPPORTED;
   if (static_cast<double>(B) * N * H * D * 2 >= 1099511627776.0) return FA_ERR_UNSUPPORTED;
-  if (B * H * ((N + kTile - 1) / kTile * kTile) / 8 >= INT32_MAX) return FA_ERR_UNSUPPORTED;  // preprocess grid
+  // preprocess grid: B N H / 16 row blocks plus B H (Npad - N) / 256 pad blocks stay below 2^31
+  if (B * H * ((N + kTile - 1) / kTile * kTile) / 15 >= INT32_MAX) return FA_ERR_UNSUPPORTED;
   if (workspace_bytes < bwd_ws_bytes(B, N, H)) return FA_ERR_INVALID_ARG;
   for (const void* p : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
                         static_cast<const void*>(dv), static_cast<const void*>(lse)})
