@@ -2,6 +2,7 @@
 """Benchmark of the fused exact-attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--pass fwd|bwd]
 
 One step = one fa_fwd call over the whole workload (default: the Llama-7B-shaped
 causal forward, B=4 H=32 N=2048 D=128 bf16). Prints ONE JSON line on rank 0.
@@ -19,6 +20,12 @@ causal forward, B=4 H=32 N=2048 D=128 bf16). Prints ONE JSON line on rank 0.
              committed ncu summary when it matches the current kernel source.
   cpu_baseline  the fp64 oracle on a bounded row sample, on the host cores
              (rank 0 at N=1 only); the same rows double as a parity check.
+
+--pass bwd times the backward instead (one step = one fa_bwd call: the D/LSE
+preprocess, the dQ kernel and the dK/dV kernel), counted as 2.5x the forward's
+flops (five N x N x D products against the forward's two); its e2e copies q,
+k, v, o, lse and dO in and dQ, dK, dV out, and its cpu_baseline is the oracle's
+backward on one (batch, head) slice.
 
 With torchrun (N>1) every rank runs the full workload on its own GPU (weak
 scaling, no collective on the data path); the timing is reduced with MAX.
@@ -39,15 +46,18 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
+METRIC_BWD = "attention bwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
+BWD_FLOP_FACTOR = 2.5  # backward flops per forward flop (5 vs 2 matrix products)
 DEFAULT_WORKLOAD = "llama7b_b4h32n2048d128_causal"
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_151_b200", "csrc", f) for f in ("fa_fwd.cu", "fa_fwd_kernel.cuh", "sm100.cuh")]
+BWD_KERNEL_SOURCES = KERNEL_SOURCES + [os.path.join(ROOT, "exact_attention_151_b200", "csrc", "fa_bwd_kernel.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_PEAK_TFLOPS = 1590.0
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources or KERNEL_SOURCES:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -71,13 +81,13 @@ def measured_hbm() -> float:
         return 6650.0
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, sources=None):
     """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
         e = d.get(workload)
-        if e and e.get("kernel_source_hash") == kernel_source_hash():
+        if e and e.get("kernel_source_hash") == kernel_source_hash(sources):
             return float(e["dram_bytes_per_launch"]), e.get("how", "")
     except Exception:
         pass
@@ -235,6 +245,196 @@ def run_reference(args, w):
     return 0
 
 
+def bwd_slice_sample(w, q, k, v, dout, target_s: float, seed: int = 0):
+    """The oracle's backward on whole (b, h) slices, as many as fit in about target_s seconds (at least one)."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_151_b200.inputs import bits
+
+    rng = np.random.default_rng(seed)
+    threads = oracle.default_threads()
+    picks, refs, dt = [], [], 0.0
+    while not picks or dt < target_s * 0.5:
+        b, h = int(rng.integers(0, w.B)), int(rng.integers(0, w.H))
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        t0 = time.perf_counter()
+        refs.append(oracle.attention_backward(bits(q[sl]), bits(k[sl]), bits(v[sl]), bits(dout[sl]), w.softmax_scale,
+                                              w.causal, w.dtype, nthreads=threads))
+        dt += time.perf_counter() - t0
+        picks.append((b, h))
+        if len(picks) >= w.B * w.H:
+            break
+    return picks, refs, dt, threads
+
+
+def run_reference_bwd(args, w):
+    """The oracle's backward on the host cores, each step whole (b, h) slices (rank 0 only)."""
+    from exact_attention_151_b200.inputs import make_dout, make_qkv
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    q, k, v = make_qkv(w)
+    dout = make_dout(w)
+    per_step_target = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    slice_flops = BWD_FLOP_FACTOR * w.flops / (w.B * w.H)
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        picks, _, dt, threads = bwd_slice_sample(w, q, k, v, dout, per_step_target, seed=100 + i)
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(slice_flops * len(picks))
+    value = sum(flops) / sum(times) / 1e12
+    sample = (f"{len(picks)} whole (b,h) slice(s) of the {w.name} workload's backward per step "
+              f"(as many as fit in ~{per_step_target:.0f} s of fp64 work, at most all B*H)")
+    line = {
+        "impl": "reference", "metric": METRIC_BWD, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(workload_config(w), **{"pass": "backward"}),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_backward(args, w, dev, world, rank):
+    """Time fa_bwd (preprocess + dQ kernel + dK/dV kernel) over the whole workload."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_151_b200 as fa
+    from exact_attention_151_b200.inputs import make_dout, make_qkv
+
+    q, k, v = make_qkv(w)
+    dout = make_dout(w)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+    od, lsed = fa.fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    workspace = torch.empty(max(fa.bwd_workspace_size(w.B, w.N, w.H), 1), dtype=torch.uint8, device=dev)
+    flops = BWD_FLOP_FACTOR * w.flops
+    # bytes a backward must move at least: read q, k, v, o, dO (16-bit) and lse, write dq, dk, dv
+    min_bytes = 8 * w.B * w.N * w.H * w.D * 2 + 4 * w.B * w.H * w.N
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if min_bytes <= 126e6 else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.bwd(qd, kd, vd, od, lsed, dod, scale=w.softmax_scale, causal=w.causal, dq=dq, dk=dk, dv=dv,
+               workspace=workspace)
+
+    for _ in range(args.warmup):
+        step()
+    if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
+        raise RuntimeError("device status word reports a timeout during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(uuid) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
+        raise RuntimeError("device status word reports a timeout in the timed region")
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(launch_ms) if flush is not None else t_start.elapsed_time(t_end)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = flops * args.steps * world / (max_ms * 1e-3) / 1e12
+    avg_ms = sum(launch_ms) / len(launch_ms)
+
+    # end to end: inputs host->device, backward, gradients device->host
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
+    hosts = [t.pin_memory() for t in (q, k, v, od.cpu(), lsed.cpu(), dout)]
+    devs = [qd, kd, vd, od, lsed, dod]
+    outs_h = [torch.empty_like(q).pin_memory() for _ in range(3)]
+
+    def e2e_step():
+        for d_, h_ in zip(devs, hosts):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in zip(outs_h, (dq, dk, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = flops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
+    h2d = sum(h_.numel() * h_.element_size() for h_ in hosts)
+    d2h = sum(h_.numel() * h_.element_size() for h_ in outs_h)
+
+    if rank == 0:
+        peak, peak_sus, peak_src = measured_peak()
+        achieved = flops / (avg_ms * 1e-3) / 1e12
+        traffic, traffic_how = recorded_traffic(w.name + ":bwd", BWD_KERNEL_SOURCES)
+        line = {
+            "metric": METRIC_BWD, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": dict(workload_config(w), **{"pass": "backward", "flops_per_step": flops}),
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
+                         "frac_of_sustained_peak": achieved / peak_sus, "algorithmic_bytes": min_bytes,
+                         "traffic_source": traffic_how,
+                         "note": "per-step time covers the preprocess, dQ and dK/dV kernels"},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "clocks": clocks.summary(),
+            "gpu_launches": args.steps * 3,
+            "kernel_source_hash": kernel_source_hash(BWD_KERNEL_SOURCES),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            from tests.parity import grad_metrics, grad_passes
+
+            picks, refs, dt, threads = bwd_slice_sample(w, q, k, v, dout, args.cpu_seconds)
+            grads = [g.cpu().to(torch.float64).numpy() for g in (dq, dk, dv)]
+            worst = None
+            for (b, h), ref in zip(picks, refs):
+                sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+                m = grad_metrics([g[sl] for g in grads], ref)
+                if worst is None or max(x["rel_l2"] for x in m.values()) > max(x["rel_l2"] for x in worst.values()):
+                    worst = m
+            line["cpu_baseline"] = {
+                "value": BWD_FLOP_FACTOR * w.flops / (w.B * w.H) * len(picks) / dt / 1e12, "unit": "TFLOP/s",
+                "cores": threads, "kind": "oracle",
+                "sample": f"{len(picks)} whole (b,h) slices of the same inputs' backward, fp64, {dt:.1f} s"}
+            line["parity"] = {"worst_slice": worst, "slices": len(picks),
+                              "passes": all(grad_passes(grad_metrics([g[(slice(b, b + 1), slice(None), slice(h, h + 1))]
+                                                                      for g in grads], ref), w.dtype)
+                                            for (b, h), ref in zip(picks, refs))}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def workload_config(w):
     extra = {} if is_square(w) else {"Nk": w.n_keys, "Hkv": w.kv_heads, "causal_alignment": "bottom-right"}
     if w.splitkv:
@@ -256,6 +456,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -263,7 +464,12 @@ def main():
     from exact_attention_151_b200.inputs import WORKLOADS
 
     w = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.which == "bwd":
+        if not is_square(w) or w.splitkv:
+            raise SystemExit("--pass bwd needs a square self-attention workload")
+        if args.impl == "reference":
+            return run_reference_bwd(args, w)
+    elif args.impl == "reference":
         return run_reference(args, w)
 
     import numpy as np
@@ -283,6 +489,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
+    if args.which == "bwd":
+        return run_backward(args, w, dev, world, rank)
 
     q, k, v = make_qkv(w)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
