@@ -403,7 +403,8 @@ def run_backward(args, w, dev, world, rank):
                          "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
                          "frac_of_sustained_peak": achieved / peak_sus, "algorithmic_bytes": min_bytes,
                          "traffic_source": traffic_how,
-                         "note": "per-step time covers the preprocess, dQ and dK/dV kernels"},
+                         "note": "achieved and frac: the whole step (preprocess, dQ and dK/dV kernels); traffic: the "
+                                 "dominant dK/dV kernel's DRAM bytes per launch"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "clocks": clocks.summary(),
