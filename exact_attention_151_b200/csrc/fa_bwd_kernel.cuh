@@ -7,7 +7,7 @@
 //   dV = P^T dO,   dP = dO V^T,   dQ = scale dS K,   dK = scale dS^T Q.
 //
 // Three kernels, no atomics (deterministic):
-//   fa_bwd_prep_kernel   D_i and LSE_i log2(e) into a workspace padded to
+//   fa_bwd_prep_kernel   -D_i and -LSE_i log2(e) into a workspace padded to
 //                        whole 128-row tiles (pad rows: D = 0, LSE = +inf, so
 //                        their weights are exactly 0);
 //   fa_bwd_kernel<.., KV_SIDE = false>  one CTA per (128-query tile, b, h):
@@ -70,8 +70,9 @@ struct Cfg {
   static constexpr int kBarDone = kBarB + 2;          // last accumulating MMA finished
   static constexpr int kBarDrain = kBarDone + 1;
   static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kWsOff = kBarOff + 128;        // key side: per compute warp -LSE log2(e), -D of 64 queries
-  static constexpr int kMiscOff = kWsOff + 8 * 512;
+  static constexpr int kWsOff = kBarOff + 128;        // key side, per stage: -LSE log2(e) and -D of the 128 queries
+  static constexpr int kWsBytes = 2 * 128 * 4;
+  static constexpr int kMiscOff = kWsOff + kStages * kWsBytes;
   static_assert(kNumBars * 8 <= 128, "barrier area");
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -83,8 +84,8 @@ struct Cfg {
 };
 
 struct Params {
-  const float* ws_d;    // [B*H, Npad]: D_i = dO_i . O_i (0 on pad rows)
-  const float* ws_l;    // [B*H, Npad]: LSE_i * log2(e) (+inf on pad rows)
+  const float* ws_d;    // [B*H, Npad]: -D_i = -dO_i . O_i (0 on pad rows)
+  const float* ws_l;    // [B*H, Npad]: -LSE_i * log2(e) (-inf on pad rows)
   uint16_t* out0;       // query side: dQ;   key side: dK
   uint16_t* out1;       // key side: dV
   int N, H, BH, Npad, n_tiles;
@@ -94,10 +95,10 @@ struct Params {
   unsigned long long wait_limit_ns;
 };
 
-// D_i and LSE_i log2(e) per row into the tile-padded workspace. Blocks below
-// n_real_blocks read O and dO in memory order ([B, N, H, D] rows, D / 8
-// threads per row, 16-byte loads); the rest fill the pad rows (D = 0,
-// LSE = +inf).
+// -D_i and -LSE_i log2(e) per row into the tile-padded workspace (negated:
+// the kernels add them). Blocks below n_real_blocks read O and dO in memory
+// order ([B, N, H, D] rows, D / 8 threads per row, 16-byte loads); the rest
+// fill the pad rows (D = 0, LSE = +inf).
 template <int D, bool FP16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __restrict__ o,
                                                           const uint16_t* __restrict__ dout,
@@ -130,8 +131,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
       const int64_t bi = row / H;
       const int i = static_cast<int>(bi % N);
       const int64_t bh = (bi / N) * H + h;
-      ws_d[bh * Npad + i] = acc;
-      ws_l[bh * Npad + i] = lse[bh * N + i] * 1.44269504088896340736f;
+      ws_d[bh * Npad + i] = -acc;
+      ws_l[bh * Npad + i] = -lse[bh * N + i] * 1.44269504088896340736f;
     }
   } else {
     const int pad = Npad - N;
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
     if (pad > 0 && p < static_cast<int64_t>(B) * H * pad) {
       const int64_t idx = (p / pad) * Npad + N + p % pad;
       ws_d[idx] = 0.f;
-      ws_l[idx] = INFINITY;
+      ws_l[idx] = -INFINITY;
     }
   }
 }
@@ -249,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto x_smem = [&](int i) { return sbase + C::kXOff + i * C::kTileBytes; };
   auto y_smem = [&](int s, int i) { return sbase + C::kYOff + (2 * s + i) * C::kTileBytes; };
   auto bar = [&](int i) { return sbase + C::kBarOff + 8 * i; };
+  auto ws_stage = [&](int s) { return sbase + C::kWsOff + s * C::kWsBytes; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
@@ -330,10 +332,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           !warp_wait_bar(bar(C::kBarYEmpty + s), static_cast<uint32_t>(((t / C::kStages) & 1) ^ 1), wc))
         break;
       const int row = row0 + (t_first + t) * kTile;
-      mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes);
+      mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + (KV_SIDE ? C::kWsBytes : 0));
       for (int hf = 0; hf < C::kHalves; ++hf) {
         tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, h, row, bar(C::kBarYFull + s));
         tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, h, row, bar(C::kBarYFull + s));
+      }
+      if constexpr (KV_SIDE) {
+        // this query tile's -LSE log2(e) and -D ride with Q_t and dO_t
+        const int64_t ws_row = static_cast<int64_t>(bh) * prm.Npad + (t_first + t) * kTile;
+        bulk_load_elect(ws_stage(s), prm.ws_l + ws_row, kTile * 4, bar(C::kBarYFull + s));
+        bulk_load_elect(ws_stage(s) + kTile * 4, prm.ws_d + ws_row, kTile * 4, bar(C::kBarYFull + s));
       }
       issued = t + 1;
     }
@@ -458,12 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* ws_l = prm.ws_l + static_cast<int64_t>(bh) * prm.Npad;
     float nl_row = 0.f, nd_row = 0.f;
     if constexpr (!KV_SIDE) {
-      nl_row = -ws_l[r_abs];
-      nd_row = -ws_d[r_abs];
+      nl_row = ws_l[r_abs];
+      nd_row = ws_d[r_abs];
     }
-    // key side: this warp's copy of -LSE log2(e) and -D for its 64 query columns
-    float* nl_col = reinterpret_cast<float*>(smem + C::kWsOff) + warp * 128;
-    float* nd_col = nl_col + 64;
     const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
     const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
     const uint32_t t_ds = KV_SIDE ? t_dp : tmem + lane_base + C::kColAcc1 + 32 * wg;
@@ -472,16 +477,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int cbase = (t_first + t) * kTile;  // first column (key, or query) of this tile
       const int first_col = cbase + 64 * wg;
       const uint32_t ph = static_cast<uint32_t>(t & 1);
-      if constexpr (KV_SIDE) {
-        __syncwarp();  // every lane is done with the previous tile's values
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          nl_col[i * 32 + lane] = -ws_l[first_col + i * 32 + lane];
-          nd_col[i * 32 + lane] = -ws_d[first_col + i * 32 + lane];
-        }
-        __syncwarp();
-      }
+      // key side: this tile's -LSE log2(e) and -D for the warpgroup's 64 query
+      // columns, in the TMA stage (the stage is released after phase B)
+      const int s = t % C::kStages;
+      const float* nl_col = reinterpret_cast<const float*>(smem + C::kWsOff + s * C::kWsBytes) + 64 * wg;
+      const float* nd_col = nl_col + kTile;
       const bool masked = (causal && cbase == tile * kTile) || cbase + kTile > N;
+      if constexpr (KV_SIDE) {
+        ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
+        if (!ok) break;
+      }
       ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
       if (!ok) break;
       tc_fence_after();
