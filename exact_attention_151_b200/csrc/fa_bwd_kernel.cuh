@@ -10,31 +10,23 @@
 //   fa_bwd_prep_kernel   -D_i and -LSE_i log2(e) into a workspace padded to
 //                        whole 128-row tiles (pad rows: D = 0, LSE = +inf, so
 //                        their weights are exactly 0);
-//   fa_bwd_kernel<.., KV_SIDE = false>  one CTA per (128-query tile, b, h):
-//                        S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - D),
-//                        dQ += dS K over the key tiles;
-//   fa_bwd_kernel<.., KV_SIDE = true>   one CTA per (128-key tile, b, h):
-//                        S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and
-//                        dS^T, dV += P^T dO and dK += dS^T Q over the query
-//                        tiles.
+//   fa_bwd_dq_kernel     one CTA per (128-query tile, b, h): S = Q K^T and
+//                        dP = dO V^T into TMEM, dS = P (dP - D), dQ += dS K
+//                        over the key tiles;
+//   fa_bwd_dkdv_kernel   one CTA per (128-key tile, b, h): S^T = K Q^T and
+//                        dP^T = V dO^T into TMEM, P^T and dS^T, dV += P^T dO
+//                        and dK += dS^T Q over the query tiles.
 //
-// One warp-specialised skeleton serves both: a TMA loader warp (the tile's
-// two fixed operands once, the streamed pair into a two-stage ring), an MMA
-// warp (converged, one elected lane issues tcgen05.mma) and two compute
-// warpgroups that split each 128-column score tile into halves (TMEM lane =
-// row, warpgroup h = columns 64h .. 64h+63). A compute thread keeps its 64
-// weights P in registers between its two phases: A reads S and forms P,
-// B reads dP and forms dS. The 16-bit MMA operands they produce go back to
-// TMEM inside the half's own columns.
-//
-// The MMA warp interleaves consecutive streamed tiles so that the tensor
-// cores work while the warpgroups compute:
-//   key side:   S(0) dP(0) | dV(t) S(t+1) dK(t) dP(t+1) | ...
-//   query side: S(0) dP(0) | S(t+1) dQ(t) dP(t+1) | ...
-// Each accumulating product is issued per half, as soon as that half's
-// operand is in TMEM. Score products keep N = 128: the tensor cores read both
-// operands of a shared-memory product from shared memory, and at N = 64 that
-// read, not the math, sets the pace.
+// Both are warp-specialised: a TMA loader warp (the tile's two fixed operands
+// once, the streamed ones through rings), an MMA warp (converged, one elected
+// lane issues tcgen05.mma) and two compute warpgroups that split each
+// 128-column score tile into halves (TMEM lane = row, warpgroup h = columns
+// 64h .. 64h+63). A compute thread keeps its 64 weights P in registers
+// between its two phases: A reads S and forms P, B reads dP and forms dS. The
+// 16-bit MMA operands they produce go back to TMEM inside the half's own
+// columns. Score products keep N = 128: the tensor cores read both operands
+// of a shared-memory product from shared memory, and at N = 64 that read,
+// not the math, sets the pace.
 #pragma once
 
 #include <cuda.h>
@@ -76,9 +68,7 @@ struct Cfg {
   static_assert(kNumBars * 8 <= 128, "barrier area");
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  // TMEM columns: scores (S or S^T), dP (or dP^T), accumulators. Key side:
-  // acc0 = dK, acc1 = dV. Query side: acc0 = dQ, and dS (16-bit pairs, 32
-  // columns per half) at acc1.
+  // TMEM columns: S^T, dP^T, accumulators acc0 = dK, acc1 = dV.
   static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
   static_assert(256 + 2 * D <= 512, "TMEM budget");
 };
@@ -150,7 +140,9 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
 // per row (query side, `nl_row`) or per column from shared memory (key side,
 // `nl_col`). MASKED tiles (the causal diagonal or the ragged tail) zero the
 // invisible entries through the exponent and use the MUFU exp only; other
-// tiles send every fourth pair through the FMA-pipe polynomial. With PACK the
+// tiles send every second pair through the FMA-pipe polynomial (the
+// backward's exp work per tile is MUFU-bound at one exp unit per SM
+// sub-partition; half on the FMA pipe measured fastest of 25/37.5/50%). With PACK the
 // 16-bit weights are stored to the half's first 32 columns (key side: P^T).
 template <bool FP16, bool KV_SIDE, bool MASKED, bool PACK>
 __device__ __forceinline__ void phase_a(uint32_t t_s, float c, float nl_row, const float* nl_col, int first_col,
@@ -189,7 +181,7 @@ __device__ __forceinline__ void phase_a(uint32_t t_s, float c, float nl_row, con
         x.y = v1 ? x.y : -INFINITY;
         pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       } else {
-        if (emulated_pair(ch * 16 + q)) {
+        if ((q & 1) == 1) {
           pp = exp2_poly2(x);
         } else {
           pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
@@ -234,15 +226,17 @@ __device__ __forceinline__ void phase_b(uint32_t t_dp, uint32_t t_out, float nd_
   }
 }
 
-// KV_SIDE = false: tile of 128 queries; X1 = Q, X2 = dO fixed, stream (K_t, V_t)
-//   over key tiles t = 0 .. last; out0 = dQ.
-// KV_SIDE = true:  tile of 128 keys; X1 = K, X2 = V fixed, stream (Q_t, dO_t)
-//   over query tiles t = first .. n_tiles-1; out0 = dK, out1 = dV.
-template <int D, bool FP16, bool KV_SIDE>
+// Key side: a tile of 128 keys; X1 = K, X2 = V stay in shared memory, (Q_t,
+// dO_t) stream over query tiles t = first .. n_tiles-1 through a two-stage
+// ring, each stage with the tile's -LSE log2(e) and -D; out0 = dK, out1 = dV.
+// TMEM holds one S^T / dP^T pair beside the two accumulators, so the MMA warp
+// interleaves consecutive tiles, S(0) dP(0) | dV(t) S(t+1) dK(t) dP(t+1) | ...,
+// issuing each accumulating product per half as soon as that half is in TMEM.
+template <int D, bool FP16>
 __global__ void __launch_bounds__(kThreads, 1)
-    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_x2,
-                  const __grid_constant__ CUtensorMap tm_y1, const __grid_constant__ CUtensorMap tm_y2,
-                  const Params prm) {
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ CUtensorMap tm_x2,
+                       const __grid_constant__ CUtensorMap tm_y1, const __grid_constant__ CUtensorMap tm_y2,
+                       const Params prm) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -258,11 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
   const int N = prm.N;
   const int causal = prm.causal;
-  // CTA -> (bh, tile). Causal work per tile is uneven (query tile i streams
-  // i + 1 key tiles; key tile j streams n_tiles - j query tiles): CTAs go in
-  // groups of kGroup heads, heaviest tiles first within a group, so the last
-  // wave holds the short ones and a group's K/V (or Q/dO) stay L2-resident.
-  // Non-causal: head-major.
+  // CTA -> (bh, key tile). Causal work per tile is uneven (key tile j streams
+  // n_tiles - j query tiles): CTAs go in groups of kGroup heads, heaviest
+  // tiles first within a group, so the last wave holds the short ones and a
+  // group's Q/dO stay L2-resident. Non-causal: head-major.
   int tile, bh;
   if (causal) {
     const int per_group = kGroup * prm.n_tiles;
@@ -271,17 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gsize = min(kGroup, prm.BH - g * kGroup);
     const int level = r / gsize;
     bh = g * kGroup + r % gsize;
-    tile = KV_SIDE ? level : prm.n_tiles - 1 - level;
+    tile = level;
   } else {
     tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
     bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
   }
   const int b = bh / prm.H, h = bh % prm.H;
-  // streamed tiles: query side: keys 0 .. (causal ? tile : n_tiles-1);
-  //                 key side:   queries (causal ? tile : 0) .. n_tiles-1
-  const int t_first = KV_SIDE ? (causal ? tile : 0) : 0;
-  const int t_last = KV_SIDE ? prm.n_tiles - 1 : (causal ? tile : prm.n_tiles - 1);
-  const int n_t = t_last - t_first + 1;
+  // streamed query tiles (causal ? tile : 0) .. n_tiles-1
+  const int t_first = causal ? tile : 0;
+  const int n_t = prm.n_tiles - t_first;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarX), 1);
@@ -332,12 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           !warp_wait_bar(bar(C::kBarYEmpty + s), static_cast<uint32_t>(((t / C::kStages) & 1) ^ 1), wc))
         break;
       const int row = row0 + (t_first + t) * kTile;
-      mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + (KV_SIDE ? C::kWsBytes : 0));
+      mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + C::kWsBytes);
       for (int hf = 0; hf < C::kHalves; ++hf) {
         tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, h, row, bar(C::kBarYFull + s));
         tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, h, row, bar(C::kBarYFull + s));
       }
-      if constexpr (KV_SIDE) {
+      {
         // this query tile's -LSE log2(e) and -D ride with Q_t and dO_t
         const int64_t ws_row = static_cast<int64_t>(bh) * prm.Npad + (t_first + t) * kTile;
         bulk_load_elect(ws_stage(s), prm.ws_l + ws_row, kTile * 4, bar(C::kBarYFull + s));
@@ -393,54 +384,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool more = t + 1 < n_t;
       const uint32_t ph = static_cast<uint32_t>(t & 1);
       const uint32_t ph_next = static_cast<uint32_t>(((t + 1) / C::kStages) & 1);
-      if constexpr (KV_SIDE) {
-        // dV += P^T dO per half as each warpgroup publishes its P^T
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
-          if (ok) {
-            tc_fence_after();
-            issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, s, hf, t == 0 && hf == 0);
-          }
-        }
-        if (!ok) break;
-        // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
-        if (more) {
-          ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
-          if (!ok) break;
+      // dV += P^T dO per half as each warpgroup publishes its P^T
+      for (int hf = 0; hf < 2 && ok; ++hf) {
+        ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
+        if (ok) {
           tc_fence_after();
-          issue_score(0, (t + 1) % C::kStages, C::kColS);
-          mma_commit_elect(bar(C::kBarSFull));
+          issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, s, hf, t == 0 && hf == 0);
         }
-        // dK += dS^T Q per half
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
-          if (ok) {
-            tc_fence_after();
-            issue_acc(C::kColAcc0, C::kColDP + 64 * hf, 0, s, hf, t == 0 && hf == 0);
-          }
-        }
-        if (!ok) break;
-      } else {
-        // both warpgroups have read S: the next tile's S may overwrite it
-        ok = warp_wait_bar(bar(C::kBarA), ph, wc) && warp_wait_bar(bar(C::kBarA + 1), ph, wc);
-        if (!ok) break;
-        if (more) {
-          ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
-          if (!ok) break;
-          tc_fence_after();
-          issue_score(0, (t + 1) % C::kStages, C::kColS);
-          mma_commit_elect(bar(C::kBarSFull));
-        }
-        // dQ += dS K per half
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
-          if (ok) {
-            tc_fence_after();
-            issue_acc(C::kColAcc0, C::kColAcc1 + 32 * hf, 0, s, hf, t == 0 && hf == 0);
-          }
-        }
-        if (!ok) break;
       }
+      if (!ok) break;
+      // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
+      if (more) {
+        ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_score(0, (t + 1) % C::kStages, C::kColS);
+        mma_commit_elect(bar(C::kBarSFull));
+      }
+      // dK += dS^T Q per half
+      for (int hf = 0; hf < 2 && ok; ++hf) {
+        ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
+        if (ok) {
+          tc_fence_after();
+          issue_acc(C::kColAcc0, C::kColDP + 64 * hf, 0, s, hf, t == 0 && hf == 0);
+        }
+      }
+      if (!ok) break;
       if (t + C::kStages < n_t) mma_commit_elect(bar(C::kBarYEmpty + s));
       if (more) {
         // dP of the next tile (after the accumulating products that read this tile's dS)
@@ -464,14 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = prm.scale_log2;
     const float* ws_d = prm.ws_d + static_cast<int64_t>(bh) * prm.Npad;
     const float* ws_l = prm.ws_l + static_cast<int64_t>(bh) * prm.Npad;
-    float nl_row = 0.f, nd_row = 0.f;
-    if constexpr (!KV_SIDE) {
-      nl_row = ws_l[r_abs];
-      nd_row = ws_d[r_abs];
-    }
+    const float nl_row = 0.f, nd_row = 0.f;  // per-column values on this side
     const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
     const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
-    const uint32_t t_ds = KV_SIDE ? t_dp : tmem + lane_base + C::kColAcc1 + 32 * wg;
+    const uint32_t t_ds = t_dp;  // dS^T pairs over the first half of this half of dP^T
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
       const int cbase = (t_first + t) * kTile;  // first column (key, or query) of this tile
@@ -483,26 +448,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* nl_col = reinterpret_cast<const float*>(smem + C::kWsOff + s * C::kWsBytes) + 64 * wg;
       const float* nd_col = nl_col + kTile;
       const bool masked = (causal && cbase == tile * kTile) || cbase + kTile > N;
-      if constexpr (KV_SIDE) {
-        ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
-        if (!ok) break;
-      }
+      ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
+      if (!ok) break;
       ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
       if (!ok) break;
       tc_fence_after();
       float p[64];
       if (masked) {
-        phase_a<FP16, KV_SIDE, true, KV_SIDE>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
+        phase_a<FP16, true, true, true>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
       } else {
-        phase_a<FP16, KV_SIDE, false, KV_SIDE>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
+        phase_a<FP16, true, false, true>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
       }
-      if constexpr (KV_SIDE) tmem_wait_st();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::kBarA + wg));
       ok = warp_wait_bar(bar(C::kBarDPFull), ph, wc);
       if (!ok) break;
       tc_fence_after();
-      phase_b<FP16, KV_SIDE>(t_dp, t_ds, nd_row, nd_col, p);
+      phase_b<FP16, true>(t_dp, t_ds, nd_row, nd_col, p);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::kBarB + wg));
@@ -510,16 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
     if (ok) {
       tc_fence_after();
-      // key side: warpgroup 0 writes dK (scaled), warpgroup 1 dV; query side:
-      // warpgroup h writes dQ columns h D/2 .. (scaled)
+      // warpgroup 0 writes dK (scaled), warpgroup 1 dV
       const bool row_valid = r_abs < N;
-      uint16_t* dst_row = (KV_SIDE && wg == 1 ? prm.out1 : prm.out0) +
-                          ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
-      const float mul = (KV_SIDE && wg == 1) ? 1.f : prm.scale;
-      constexpr int kCols = KV_SIDE ? D : D / 2;
-      const uint32_t acc = tmem + lane_base + (KV_SIDE ? (wg == 0 ? C::kColAcc0 : C::kColAcc1)
-                                                       : C::kColAcc0 + wg * (D / 2));
-      const int col0 = KV_SIDE ? 0 : wg * (D / 2);
+      uint16_t* dst_row = (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
+      const float mul = wg == 1 ? 1.f : prm.scale;
+      constexpr int kCols = D;
+      const uint32_t acc = tmem + lane_base + (wg == 0 ? C::kColAcc0 : C::kColAcc1);
+      const int col0 = 0;
 #pragma unroll
       for (int q = 0; q < kCols / 32; ++q) {
         uint32_t a[32];
@@ -531,6 +491,302 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul);
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + col0 + q * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Query side with a double-buffered score tile. One CTA per (128-query tile,
+// b, h); Q and dO stay in shared memory, K_t streams through a three-stage
+// ring and V_t through a two-stage ring. TMEM: S(t) in buffer t % 2 (columns
+// 0 and 128), dP at 256, dQ at 384; dS(t) is written back over the first half
+// of each warpgroup's columns of its own S buffer. The MMA warp waits once per
+// streamed tile, for both warpgroups' dS(t), and then issues
+//   dP(t+1), dQ(t), S(t+2)
+// back to back, so the score product two tiles ahead is already in TMEM when
+// the warpgroups need it.
+template <int D>
+struct CfgQ {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kSlabBytes = 128 * 128;
+  static constexpr int kTileBytes = kHalves * kSlabBytes;
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 2;
+  static constexpr int kXOff = 0;                                // Q, dO
+  static constexpr int kKOff = kXOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kBarX = 0;
+  static constexpr int kBarKFull = 1;                             // [kKStages]
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;         // [kKStages]
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;         // [kVStages]
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;         // [kVStages]
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;         // [2] S buffer b holds S(t), t % 2 == b
+  static constexpr int kBarDPFull = kBarSFull + 2;
+  static constexpr int kBarB = kBarDPFull + 1;                    // [2] warpgroup h wrote dS(t) (128 arrivals)
+  static constexpr int kBarDone = kBarB + 2;
+  static constexpr int kBarDrain = kBarDone + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static_assert(kNumBars * 8 <= 256, "barrier area");
+  static constexpr int kMiscOff = kBarOff + 256;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static constexpr uint32_t kColS0 = 0, kColDP = 256, kColAcc = 384;
+  static_assert(384 + D <= 512, "TMEM budget");
+};
+
+template <int D, bool FP16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const Params prm) {
+  using C = CfgQ<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto x_smem = [&](int i) { return sbase + C::kXOff + i * C::kTileBytes; };
+  auto k_smem = [&](int s) { return sbase + C::kKOff + s * C::kTileBytes; };
+  auto v_smem = [&](int s) { return sbase + C::kVOff + s * C::kTileBytes; };
+  auto bar = [&](int i) { return sbase + C::kBarOff + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int N = prm.N;
+  const int causal = prm.causal;
+  // CTA -> (bh, query tile): causal in groups of kGroup heads, heaviest
+  // (latest) query tiles first; non-causal head-major.
+  int tile, bh;
+  if (causal) {
+    const int per_group = kGroup * prm.n_tiles;
+    const int g = static_cast<int>(blockIdx.x) / per_group;
+    const int r = static_cast<int>(blockIdx.x) % per_group;
+    const int gsize = min(kGroup, prm.BH - g * kGroup);
+    bh = g * kGroup + r % gsize;
+    tile = prm.n_tiles - 1 - r / gsize;
+  } else {
+    tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
+    bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
+  }
+  const int b = bh / prm.H, h = bh % prm.H;
+  const int n_t = causal ? tile + 1 : prm.n_tiles;  // key tiles 0 .. n_t-1
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::kBarX), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::kBarSFull + i), 1);
+      mbar_init(bar(C::kBarB + i), 128);
+    }
+    mbar_init(bar(C::kBarDPFull), 1);
+    mbar_init(bar(C::kBarDone), 1);
+    mbar_init(bar(C::kBarDrain), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMma) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, prm.wait_limit_ns};
+  const int row0 = b * N;
+
+  if (warp == kLoad) {
+    // ------------------------------------------------------------ loader (converged warp)
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    __syncwarp();
+    mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
+    for (int hf = 0; hf < C::kHalves; ++hf) {
+      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
+      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_do, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
+    }
+    int nk = 0, nv = 0;  // K and V tiles issued
+    for (int t = 0; t < n_t; ++t) {
+      const int row = row0 + t * kTile;
+      const int sk = t % C::kKStages;
+      if (t >= C::kKStages &&
+          !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((t / C::kKStages) & 1) ^ 1), wc))
+        break;
+      mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, row, bar(C::kBarKFull + sk));
+      nk = t + 1;
+      const int sv = t % C::kVStages;
+      if (t >= C::kVStages &&
+          !warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((t / C::kVStages) & 1) ^ 1), wc))
+        break;
+      mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, row, bar(C::kBarVFull + sv));
+      nv = t + 1;
+    }
+    // let the copies this warp issued land before shared memory is released
+    drain_wait(bar(C::kBarX), 0);
+    for (int s = 0; s < C::kKStages && s < nk; ++s) {
+      const int tl = s + ((nk - 1 - s) / C::kKStages) * C::kKStages;
+      drain_wait(bar(C::kBarKFull + s), static_cast<uint32_t>((tl / C::kKStages) & 1));
+    }
+    for (int s = 0; s < C::kVStages && s < nv; ++s) {
+      const int tl = s + ((nv - 1 - s) / C::kVStages) * C::kVStages;
+      drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((tl / C::kVStages) & 1));
+    }
+  } else if (warp == kMma) {
+    // ------------------------------------------------------------ MMA issue (converged warp)
+    constexpr uint32_t idesc_score = instr_desc_f16(kTile, kTile, FP16, false);
+    constexpr uint32_t idesc_acc = instr_desc_f16(kTile, D, FP16, true);
+    constexpr uint64_t kTileStep = C::kTileBytes >> 4;
+    const uint64_t q_desc = smem_desc_sw128(x_smem(0), 16, 1024);  // K-major
+    const uint64_t do_desc = smem_desc_sw128(x_smem(1), 16, 1024);
+    const uint64_t k_desc0 = smem_desc_sw128(k_smem(0), 16, 1024);
+    const uint64_t v_desc0 = smem_desc_sw128(v_smem(0), 16, 1024);
+    const uint64_t k_mn0 = smem_desc_sw128(k_smem(0), C::kSlabBytes, 1024);  // K_t as MN-major B of dQ += dS K
+    // X Y^T into TMEM column `col`, K = D in steps of 16 (both operands K-major)
+    auto issue_score = [&](uint64_t a, uint64_t bb, uint32_t col) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
+        mma_ss_elect(tmem + col, a + off, bb + off, idesc_score, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_s = [&](int t) {  // S(t) = Q K_t^T into buffer t % 2
+      issue_score(q_desc, k_desc0 + static_cast<uint64_t>(t % C::kKStages) * kTileStep, C::kColS0 + 128 * (t & 1));
+      mma_commit_elect(bar(C::kBarSFull + (t & 1)));
+    };
+    auto issue_dp = [&](int t) {  // dP(t) = dO V_t^T
+      issue_score(do_desc, v_desc0 + static_cast<uint64_t>(t % C::kVStages) * kTileStep, C::kColDP);
+      mma_commit_elect(bar(C::kBarDPFull));
+    };
+    bool ok = warp_wait_bar(bar(C::kBarX), 0, wc) && warp_wait_bar(bar(C::kBarKFull), 0, wc);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+      ok = warp_wait_bar(bar(C::kBarVFull), 0, wc);
+    }
+    if (ok) {
+      tc_fence_after();
+      issue_dp(0);
+      if (n_t > 1) {
+        ok = warp_wait_bar(bar(C::kBarKFull + 1), 0, wc);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
+        }
+      }
+    }
+    for (int t = 0; ok && t < n_t; ++t) {
+      const uint32_t ph = static_cast<uint32_t>(t & 1);
+      // both warpgroups have read dP(t) and written dS(t) into S buffer t % 2
+      ok = warp_wait_bar(bar(C::kBarB), ph, wc) && warp_wait_bar(bar(C::kBarB + 1), ph, wc);
+      if (!ok) break;
+      tc_fence_after();
+      mma_commit_elect(bar(C::kBarVEmpty + t % C::kVStages));  // V_t: its reader dP(t) is done
+      if (t + 1 < n_t) {
+        ok = warp_wait_bar(bar(C::kBarVFull + (t + 1) % C::kVStages), static_cast<uint32_t>(((t + 1) / C::kVStages) & 1),
+                           wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dp(t + 1);
+      }
+      // dQ += dS(t) K_t: A = dS pairs in S buffer t % 2 (warpgroup h: columns 64h ..), B = K_t MN-major
+      const uint64_t kb = k_mn0 + static_cast<uint64_t>(t % C::kKStages) * kTileStep;
+      const uint32_t a0 = C::kColS0 + 128 * (t & 1);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        mma_ts_elect(tmem + C::kColAcc, tmem + a0 + 64 * (kk / 4) + 8 * (kk % 4), kb + static_cast<uint64_t>(kk * (2048 >> 4)),
+                     idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit_elect(bar(C::kBarKEmpty + t % C::kKStages));  // K_t: last reader issued
+      if (t + 2 < n_t) {
+        ok = warp_wait_bar(bar(C::kBarKFull + (t + 2) % C::kKStages), static_cast<uint32_t>(((t + 2) / C::kKStages) & 1),
+                           wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(t + 2);  // into buffer t % 2, after dQ(t) has read dS(t) from it (in order)
+      }
+      if (t == n_t - 1) mma_commit_elect(bar(C::kBarDone));
+    }
+    if (!ok) {
+      mma_commit_elect(bar(C::kBarDrain));
+      drain_wait(bar(C::kBarDrain), 0);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
+    const int wg = warp / 4;                  // column half of every score tile
+    const int qd = warp % 4;                  // TMEM lane quadrant
+    const int row = qd * 32 + lane;
+    const int r_abs = tile * kTile + row;     // this thread's query
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const float c = prm.scale_log2;
+    const float nl_row = prm.ws_l[static_cast<int64_t>(bh) * prm.Npad + r_abs];
+    const float nd_row = prm.ws_d[static_cast<int64_t>(bh) * prm.Npad + r_abs];
+    bool ok = true;
+    for (int t = 0; t < n_t; ++t) {
+      const int first_col = t * kTile + 64 * wg;  // first key of this warpgroup's half
+      const uint32_t t_s = tmem + lane_base + C::kColS0 + 128 * (t & 1) + 64 * wg;
+      const bool masked = (causal && t == tile) || (t + 1) * kTile > N;
+      ok = warp_wait_bar(bar(C::kBarSFull + (t & 1)), static_cast<uint32_t>((t >> 1) & 1), wc);
+      if (!ok) break;
+      tc_fence_after();
+      float p[64];
+      if (masked) {
+        phase_a<FP16, false, true, false>(t_s, c, nl_row, nullptr, first_col, r_abs, N, causal, p);
+      } else {
+        phase_a<FP16, false, false, false>(t_s, c, nl_row, nullptr, first_col, r_abs, N, causal, p);
+      }
+      ok = warp_wait_bar(bar(C::kBarDPFull), static_cast<uint32_t>(t & 1), wc);
+      if (!ok) break;
+      tc_fence_after();
+      // dS pairs over the first 32 columns of this half of S(t) (read above)
+      phase_b<FP16, false>(tmem + lane_base + C::kColDP + 64 * wg, t_s, nd_row, nullptr, p);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarB + wg));
+    }
+    if (ok) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
+    if (ok) {
+      tc_fence_after();
+      // warpgroup h writes dQ columns h D/2 .. (scaled)
+      const bool row_valid = r_abs < N;
+      uint16_t* dst_row = prm.out0 + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D + wg * (D / 2);
+      const uint32_t acc = tmem + lane_base + C::kColAcc + wg * (D / 2);
+#pragma unroll
+      for (int q = 0; q < D / 64; ++q) {
+        uint32_t a[32];
+        tmem_ld32(acc + q * 32, a);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * prm.scale, __uint_as_float(a[2 * k + 1]) * prm.scale);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }

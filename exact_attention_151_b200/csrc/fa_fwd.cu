@@ -313,13 +313,13 @@ size_t bwd_ws_bytes(int64_t B, int64_t N, int64_t H) {
 template <int D, bool FP16, bool KV_SIDE>
 fa_status bwd_launch(int dev, const CUtensorMap& x1, const CUtensorMap& x2, const CUtensorMap& y1,
                      const CUtensorMap& y2, const bwd::Params& prm, int64_t grid, cudaStream_t stream) {
-  using C = bwd::Cfg<D>;
-  auto kernel = bwd::fa_bwd_kernel<D, FP16, KV_SIDE>;
+  constexpr int kSmem = KV_SIDE ? bwd::Cfg<D>::kSmemBytes : bwd::CfgQ<D>::kSmemBytes;
+  auto kernel = KV_SIDE ? bwd::fa_bwd_dkdv_kernel<D, FP16> : bwd::fa_bwd_dq_kernel<D, FP16>;
   const unsigned bit = 1u << (4 + (D == 128 ? 4 : 0) + (FP16 ? 2 : 0) + (KV_SIDE ? 1 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(g_devices[dev].configured & bit)) {
-      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
       if (e != cudaSuccess) {
         set_error("cudaFuncSetAttribute(backward)", e);
         cudaGetLastError();
@@ -328,7 +328,7 @@ fa_status bwd_launch(int dev, const CUtensorMap& x1, const CUtensorMap& x2, cons
       g_devices[dev].configured |= bit;
     }
   }
-  kernel<<<static_cast<unsigned>(grid), bwd::kThreads, C::kSmemBytes, stream>>>(x1, x2, y1, y2, prm);
+  kernel<<<static_cast<unsigned>(grid), bwd::kThreads, kSmem, stream>>>(x1, x2, y1, y2, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(KV_SIDE ? "backward dK/dV launch" : "backward dQ launch", e);
