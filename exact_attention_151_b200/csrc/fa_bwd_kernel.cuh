@@ -431,8 +431,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_abs = tile * kTile + row;     // this thread's query (or key) index
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const float c = prm.scale_log2;
-    const float* ws_d = prm.ws_d + static_cast<int64_t>(bh) * prm.Npad;
-    const float* ws_l = prm.ws_l + static_cast<int64_t>(bh) * prm.Npad;
     const float nl_row = 0.f, nd_row = 0.f;  // per-column values on this side
     const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
     const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
