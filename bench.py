@@ -503,7 +503,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
     kernels_per_step = 1
     if w.splitkv:
-        n_splits, ws_bytes = fa.splitkv_plan(w.B, w.N, w.n_keys, w.H, w.D)
+        n_splits, ws_bytes = fa.splitkv_plan(w.B, w.N, w.n_keys, w.H, w.D, Hkv=w.kv_heads)
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         kernels_per_step = 2 if n_splits > 1 else 1
 

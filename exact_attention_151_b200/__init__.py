@@ -80,7 +80,7 @@ def load_library():
     lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32, i32, vp,
                                    ctypes.c_size_t, vp]
     lib.fa_fwd_splitkv.restype = i32
-    lib.fa_fwd_splitkv_plan.argtypes = [i64, i64, i64, i64, i64, i32, ctypes.POINTER(i32),
+    lib.fa_fwd_splitkv_plan.argtypes = [i64, i64, i64, i64, i64, i64, i32, ctypes.POINTER(i32),
                                         ctypes.POINTER(ctypes.c_size_t)]
     lib.fa_fwd_splitkv_plan.restype = i32
     lib.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32, i32,
@@ -228,11 +228,14 @@ def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, scale: fl
     return o, lse
 
 
-def splitkv_plan(B: int, Nq: int, Nk: int, Hq: int, D: int, num_splits: int = 0) -> tuple[int, int]:
-    """(number of key ranges, workspace bytes) fa_fwd_splitkv uses for these sizes on the current device."""
+def splitkv_plan(B: int, Nq: int, Nk: int, Hq: int, D: int, num_splits: int = 0, Hkv: int | None = None) -> tuple[int, int]:
+    """(number of key ranges, workspace bytes) fa_fwd_splitkv uses for these sizes on the current device.
+    ``Hkv`` (default Hq) selects the packed-heads grid when Nq * Hq / Hkv <= 128."""
     n = ctypes.c_int(0)
     size = ctypes.c_size_t(0)
-    st = load_library().fa_fwd_splitkv_plan(B, Nq, Nk, Hq, D, int(num_splits), ctypes.byref(n), ctypes.byref(size))
+    hkv = Hq if Hkv is None else Hkv
+    st = load_library().fa_fwd_splitkv_plan(B, Nq, Nk, Hq, hkv, D, int(num_splits), ctypes.byref(n),
+                                            ctypes.byref(size))
     if st != FA_OK:
         raise FaError(st, "fa_fwd_splitkv_plan")
     return n.value, size.value
@@ -255,7 +258,7 @@ def fwd_splitkv(q, k, v, scale: float | None = None, causal: bool = False, num_s
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     with torch.cuda.device(q.device):
-        _, need = splitkv_plan(B, Nq, Nk, Hq, D, num_splits)
+        _, need = splitkv_plan(B, Nq, Nk, Hq, D, num_splits, Hkv=Hkv)
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
         if o is None:

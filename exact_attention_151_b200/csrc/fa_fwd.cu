@@ -68,12 +68,13 @@ fa_status load_encoder() {
 }
 
 // A [rows, H, D] 16-bit tensor (a dense [B, N, H, D] tensor is B*N rows)
-// viewed as 3-D (D, H, rows), box (64, 1, 128), 128B swizzle; rows past the
-// end are zero-filled by TMA.
-fa_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t H, int64_t D, bool fp16) {
+// viewed as 3-D (D, H, rows), box (64, box_h, box_rows) (default one head by
+// 128 rows), 128B swizzle; rows past the end are zero-filled by TMA.
+fa_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t H, int64_t D, bool fp16,
+                    uint32_t box_h = 1, uint32_t box_rows = 128) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(H * D * 2)};
-  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t box[3] = {64, box_h, box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = g_encode(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -115,6 +116,7 @@ struct Shape {
   const int* cu_q;
   const int* cu_k;
   int64_t B, Nq, Nk, total_q, total_k, max_nq, Hq, Hkv, D;
+  int pack_g = 0;         // packed heads (dense, Nq * G <= 128): G = Hq / Hkv, else 0
   int n_splits = 1;       // split-KV (dense shapes): number of key ranges
   int split_tiles = 0;    // key tiles per range
   float* part_o = nullptr;
@@ -166,9 +168,11 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.total_k = static_cast<int>(sh.total_k);
   prm.Hq = static_cast<int>(sh.Hq);
   prm.Hkv = static_cast<int>(sh.Hkv);
-  prm.BH = static_cast<int>(sh.B * sh.Hq);
+  prm.BH = static_cast<int>(sh.pack_g ? sh.B * sh.Hkv : sh.B * sh.Hq);
+  prm.BHq = static_cast<int>(sh.B * sh.Hq);
+  prm.pack_g = sh.pack_g;
   prm.max_nq = static_cast<int>(sh.max_nq);
-  prm.n_blocks = static_cast<int>((sh.max_nq + kBlockRows - 1) / kBlockRows);
+  prm.n_blocks = sh.pack_g ? 1 : static_cast<int>((sh.max_nq + kBlockRows - 1) / kBlockRows);
   // Softmax runs in base 2: x = s * scale * log2(e). A zero (or subnormal)
   // factor is replaced by +-FLT_MIN: every weight then still rounds to
   // exactly 1 (|s| < 2^40 for 16-bit inputs) while masked keys keep weight 0.
@@ -182,7 +186,7 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.split_tiles = sh.split_tiles;
   prm.part_o = sh.part_o;
   prm.part_lse = sh.part_lse;
-  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * sh.B * sh.Hq * sh.n_splits;
+  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * prm.BH * sh.n_splits;
   kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -221,13 +225,22 @@ size_t splitkv_bytes(int64_t n_splits, int64_t BH, int64_t Nq, int64_t D) {
   return align256(static_cast<size_t>(n_splits * BH * Nq * D) * 4) + align256(static_cast<size_t>(n_splits * BH * Nq) * 4);
 }
 
+// Packed heads (one query tile per key/value head holds all G = Hq / Hkv query
+// heads for every query position) for dense shapes with Nq * G <= 128, G > 1.
+int64_t pack_group(int64_t Nq, int64_t Hq, int64_t Hkv) {
+  if (Hkv < 1 || Hq % Hkv != 0) return 0;
+  const int64_t g = Hq / Hkv;
+  return (g > 1 && Nq >= 1 && Nq * g <= kTile) ? g : 0;
+}
+
 // Number of key ranges: when the query side alone fills less than half the
 // SMs, as many ranges as keep the CTAs within one wave (one CTA per SM), never
 // more than the key tiles or kMaxSplits; the count is then evened so every
 // range has the same number of tiles.
-int resolve_splits(int requested, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int sm_count, int* tiles_out) {
+int resolve_splits(int requested, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int sm_count,
+                   int* tiles_out) {
   const int64_t n_kt = (Nk + kTile - 1) / kTile;
-  const int64_t base = ((Nq + kBlockRows - 1) / kBlockRows) * B * Hq;
+  const int64_t base = pack_group(Nq, Hq, Hkv) ? B * Hkv : ((Nq + kBlockRows - 1) / kBlockRows) * B * Hq;
   int64_t want = requested;
   if (want <= 0) want = (base >= sm_count / 2 || n_kt < 2) ? 1 : sm_count / base;
   want = std::max<int64_t>(1, std::min<int64_t>({want, n_kt > 0 ? n_kt : 1, kMaxSplits}));
@@ -282,17 +295,22 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   const int64_t krows = sh.total_k > 0 ? sh.total_k : 1;
   const int64_t khead = sh.total_k > 0 ? sh.Hkv : 1;
   CUtensorMap tq, tk, tv;
-  if (make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16) != FA_OK || make_tmap(&tk, kb, krows, khead, sh.D, fp16) != FA_OK ||
+  Shape shp = sh;
+  shp.pack_g = sh.cu_q == nullptr ? static_cast<int>(pack_group(sh.Nq, sh.Hq, sh.Hkv)) : 0;
+  const fa_status mq = shp.pack_g ? make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16, static_cast<uint32_t>(shp.pack_g),
+                                              static_cast<uint32_t>(sh.Nq))
+                                  : make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16);
+  if (mq != FA_OK || make_tmap(&tk, kb, krows, khead, sh.D, fp16) != FA_OK ||
       make_tmap(&tv, vb, krows, khead, sh.D, fp16) != FA_OK)
     return FA_ERR_CUDA;
   if (limit_ns == 0) limit_ns = kDefaultWaitLimitNs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (sh.D == 128) {
-    return fp16 ? launch<128, true>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold)
-                : launch<128, false>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold);
+    return fp16 ? launch<128, true>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold)
+                : launch<128, false>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold);
   }
-  return fp16 ? launch<64, true>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold)
-              : launch<64, false>(dev, tq, tk, tv, o, lse, sh, scale, causal, s, limit_ns, withhold);
+  return fp16 ? launch<64, true>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold)
+              : launch<64, false>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold);
 }
 
 Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D) {
@@ -509,10 +527,10 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   }
 }
 
-fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t D, int num_splits,
+fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, int num_splits,
                               int* splits_out, size_t* workspace_bytes) {
   try {
-    if (!splits_out || !workspace_bytes || B < 0 || Nq < 0 || Nk < 0 || Hq < 0 || num_splits < 0)
+    if (!splits_out || !workspace_bytes || B < 0 || Nq < 0 || Nk < 0 || Hq < 0 || Hkv < 0 || num_splits < 0)
       return FA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
     int dev = 0;
@@ -522,7 +540,7 @@ fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int
     }
     const int sms = dev >= 0 ? fa::device_sm_count(dev) : 148;
     int tiles = 0;
-    const int splits = fa::resolve_splits(num_splits, B, Nq, Nk, Hq, sms, &tiles);
+    const int splits = fa::resolve_splits(num_splits, B, Nq, Nk, Hq, Hkv, sms, &tiles);
     *splits_out = splits;
     *workspace_bytes = splits > 1 ? fa::splitkv_bytes(splits, B * Hq, Nq, D) : 0;
     return FA_OK;
@@ -539,7 +557,7 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
     if (num_splits < 0) return FA_ERR_INVALID_ARG;
     int splits = 1, tiles = 0;
     size_t need = 0;
-    fa_status st = fa_fwd_splitkv_plan(B < 0 ? 0 : B, Nq < 0 ? 0 : Nq, Nk < 0 ? 0 : Nk, Hq < 0 ? 0 : Hq,
+    fa_status st = fa_fwd_splitkv_plan(B < 0 ? 0 : B, Nq < 0 ? 0 : Nq, Nk < 0 ? 0 : Nk, Hq < 0 ? 0 : Hq, Hkv < 0 ? 0 : Hkv,
                                        D, num_splits, &splits, &need);
     if (st != FA_OK) return st;
     if (splits > 1) {
@@ -547,7 +565,7 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
       if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
       int dev = 0;
       cudaGetDevice(&dev);
-      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, fa::device_sm_count(dev), &tiles);
+      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, Hkv, fa::device_sm_count(dev), &tiles);
       sh.n_splits = splits;
       sh.split_tiles = tiles;
       sh.part_o = static_cast<float*>(workspace);
@@ -567,7 +585,7 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
     if (num_splits < 0 || B < 0 || Nq < 0 || Nk < 0 || Hq < 0) return FA_ERR_INVALID_ARG;
     int splits = 1;
     size_t need = 0;
-    fa_status st = fa_fwd_splitkv_plan(B, Nq, Nk, Hq, D, num_splits, &splits, &need);
+    fa_status st = fa_fwd_splitkv_plan(B, Nq, Nk, Hq, Hkv, D, num_splits, &splits, &need);
     if (st != FA_OK) return st;
     if (need > fa::kNoAllocScratchBytes) {
       std::snprintf(fa::g_last_error, sizeof(fa::g_last_error),
@@ -589,7 +607,7 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
       st = fa::noalloc_scratch_address(dev, &scratch);
       if (st != FA_OK) return st;
       int tiles = 0;
-      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, fa::device_sm_count(dev), &tiles);
+      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, Hkv, fa::device_sm_count(dev), &tiles);
       sh.n_splits = splits;
       sh.split_tiles = tiles;
       sh.part_o = static_cast<float*>(scratch);

@@ -262,6 +262,13 @@ struct Params {
   float* part_lse;
   unsigned long long wait_limit_ns;
   int withhold_v_load;
+  // Packed heads (dense shapes with Nq * G <= 128, G = Hq / Hkv > 1): one work
+  // item per (batch, key/value head); its single query tile holds the G query
+  // heads sharing that K/V head for every query position, row n G + g = query
+  // n of head hk G + g (one TMA box of (64, G, Nq)). BH then counts B * Hkv
+  // items and BHq = B * Hq query heads. 0: off.
+  int pack_g;
+  int BHq;
 };
 
 template <int D, bool FP16>
@@ -313,9 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     level = xblk % prm.n_blocks;
   }
   const int mb = causal ? (prm.n_blocks - 1 - level) : level;
-  const int b = bh / prm.Hq;
-  const int h = bh % prm.Hq;
-  const int hk = h / (prm.Hq / prm.Hkv);  // key/value head of this query head
+  const int pg = prm.pack_g;
+  const int b = pg ? bh / prm.Hkv : bh / prm.Hq;
+  const int h = pg ? (bh % prm.Hkv) * pg : bh % prm.Hq;    // (first) query head
+  const int hk = pg ? bh % prm.Hkv : h / (prm.Hq / prm.Hkv);  // key/value head
   // This sequence's rows: queries q0 .. q0+nq-1, keys k0 .. k0+nk-1.
   int q0, nq, k0, nk;
   if (prm.cu_q != nullptr) {
@@ -341,12 +349,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int delta = nk - nq;  // causal offset: query i sees keys j <= i + delta
   const int qt0 = 2 * mb;
   const int qt1 = 2 * mb + 1;
-  const bool q1_valid = qt1 < n_qt;
+  const bool q1_valid = !pg && qt1 < n_qt;
+  // smallest and largest query index held by query tile qt (packed heads:
+  // the first and the last query)
+  auto q_min = [&](int qt) -> int { return pg ? 0 : qt * kTile; };
+  auto q_max = [&](int qt) -> int { return pg ? nq - 1 : qt * kTile + kTile - 1; };
   // last key tile holding a key visible to some row of query tile qt (-1: none)
   auto last_key_tile = [&](int qt) -> int {
     if (nk == 0) return -1;
     if (!causal) return n_kt - 1;
-    const int last_key = qt * kTile + kTile - 1 + delta;
+    const int last_key = q_max(qt) + delta;
     if (last_key < 0) return -1;
     return min(n_kt - 1, last_key / kTile);
   };
@@ -406,10 +418,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_v);
       }
       __syncwarp();
-      mbar_arrive_expect_tx_elect(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
-      for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
+      if (pg) {
+        // packed heads: one (64, G, Nq) box per slab fills rows 0 .. G Nq - 1
+        mbar_arrive_expect_tx_elect(bar(C::kBarQ), C::kHalves * pg * nq * 128);
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0 + (qt0 + i) * kTile, bar(C::kBarQ));
+          tma_load_3d_elect(q_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0, bar(C::kBarQ));
+      } else {
+        mbar_arrive_expect_tx_elect(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
+        for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_3d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0 + (qt0 + i) * kTile, bar(C::kBarQ));
+      }
       const bool withhold = prm.withhold_v_load && blockIdx.x == 0;
       int nk = 0, nv = 0;  // K and V tiles issued
       for (int j = 0; j < n_kv; ++j) {
@@ -551,7 +570,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int last = wg == 0 ? last0 : last1;
     const int quarter = warp % 4;         // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int qi = qt * kTile + row;
+    // this row's query index and head (packed heads: row = n G + g)
+    const int qi = pg ? row / pg : qt * kTile + row;
+    const int hq = pg ? h + row % pg : h;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_col = tmem + lane_base + C::col_s(wg);
     const uint32_t o_col = tmem + lane_base + C::col_o(wg);
@@ -575,7 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kTile; ++k) s[k] = __uint_as_float(r[k / 32][k % 32]);
       }
       const int kbase = (jb + j) * kTile;
-      if (kbase + kTile > nk || (causal && kbase + kTile - 1 > qt * kTile + delta)) {
+      // masking is needed when some row of the tile sees only part of it: the
+      // tile runs past the keys, or past the first row's last visible key
+      if (kbase + kTile > nk || (causal && kbase + kTile - 1 > q_min(qt) + delta)) {
         // last visible column of this row in this tile (may be < 0: none)
         const int lastcol = (causal ? min(nk - 1, qi + delta) : (nk - 1)) - kbase;
 #pragma unroll
@@ -622,11 +645,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and LSE = -inf, whatever its TMEM lanes hold.
     const bool splitkv = prm.n_splits > 1;
     const int row_last_key = causal ? min(nk - 1, qi + delta) : nk - 1;
-    const bool row_valid = (wg == 0 || q1_valid) && qi < nq;
+    const bool row_valid = (wg == 0 || q1_valid) && qi < nq && (!pg || row < pg * nq);
     const bool row_has_keys = row_last_key >= 0 && (!splitkv || row_last_key >= jb * kTile);
     if (splitkv) {
       // fp32 partial result of this key range (normalised by its own sum)
-      const int64_t prow = (static_cast<int64_t>(split) * prm.BH + bh) * prm.Nq + qi;
+      const int64_t prow = (static_cast<int64_t>(split) * prm.BHq + static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi;
       float* orow = prm.part_o + prow * D;
       if (last >= 0 && ok) {
         tc_fence_after();
@@ -658,10 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         prm.part_lse[prow] = -INFINITY;
       }
     } else {
-      uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + h) * D;
+      uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + hq) * D;
       float* lse_at = prm.lse + (prm.cu_q != nullptr
-                                     ? static_cast<int64_t>(h) * prm.total_q + q0 + qi
-                                     : (static_cast<int64_t>(b) * prm.Hq + h) * prm.Nq + qi);
+                                     ? static_cast<int64_t>(hq) * prm.total_q + q0 + qi
+                                     : (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi);
       if (last >= 0 && ok) {
         tc_fence_after();
         const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;

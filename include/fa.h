@@ -155,9 +155,13 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
 /*
  * fa_fwd_splitkv_plan - number of key ranges fa_fwd_splitkv will use for
  * these sizes on the current device, and the workspace it needs in bytes
- * (0 when it uses one range). Host only; launches nothing.
+ * (0 when it uses one range). Host only; launches nothing. Hkv matters:
+ * when Nq * (Hq / Hkv) <= 128 and Hq / Hkv > 1 the forward packs the query
+ * heads that share a key/value head into one tile (one work item per K/V head
+ * instead of one per query head), and the key range count is chosen for that
+ * smaller grid.
  */
-fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t D, int num_splits,
+fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, int num_splits,
                               int* splits_out, size_t* workspace_bytes);
 
 /*

@@ -105,3 +105,31 @@ def test_inconsistent_offsets_are_reported_and_skipped():
     cu_k2 = torch.tensor([0, 10, 100], dtype=torch.int32, device=DEV)
     fa.fwd_varlen(q, k, k, cu_q2, cu_k2, 50, o=o, lse=lse)
     assert fa.status_sync() == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,Nq,Nk,Hq,Hkv,D,dtype", [
+    (2, 1, 300, 8, 2, 128, "bf16"),     # decode, 4 heads per K/V head
+    (1, 16, 1000, 32, 4, 128, "bf16"),  # 16 x 8 = 128 rows: a full packed tile
+    (3, 3, 517, 12, 3, 64, "fp16"),     # ragged: 12 rows, bottom-right causal with several queries
+    (1, 2, 64, 64, 1, 128, "bf16"),     # 64 heads on one K/V head, fewer keys than a tile
+    (2, 5, 0, 8, 4, 64, "bf16"),        # no keys: O = 0, LSE = -inf
+])
+def test_packed_heads(B, Nq, Nk, Hq, Hkv, D, dtype, causal):
+    """Nq * (Hq / Hkv) <= 128: the query heads sharing a K/V head are packed into one tile."""
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    seed = B * 1000 + Nq * 31 + Nk + Hq
+    q = _randn((B, Nq, Hq, D), seed, tdt)
+    k = _randn((B, Nk, Hkv, D), seed + 1, tdt)
+    v = _randn((B, Nk, Hkv, D), seed + 2, tdt)
+    o, lse = fa.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal)
+    assert fa.status_sync() == fa.FA_OK
+    cu_q, cu_k = np.arange(B + 1) * Nq, np.arange(B + 1) * Nk
+    o_ref, lse_ref = oracle.attention_varlen(bits(q.reshape(B * Nq, Hq, D)), bits(k.reshape(B * Nk, Hkv, D)),
+                                             bits(v.reshape(B * Nk, Hkv, D)), cu_q, cu_k, 1 / math.sqrt(D), causal,
+                                             dtype)
+    lse_g = lse.cpu().permute(1, 0, 2).reshape(Hq, B * Nq).numpy()
+    finite = np.isfinite(lse_ref)
+    assert np.all(np.isneginf(lse_g[~finite]))
+    _check(o.cpu().double().reshape(B * Nq, Hq, D).numpy(), np.where(finite, lse_g, 0.0), o_ref,
+           np.where(finite, lse_ref, 0.0))

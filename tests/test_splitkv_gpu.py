@@ -52,7 +52,7 @@ def test_splitkv_matches_oracle(B, Nq, Nk, Hq, Hkv, D, dtype, splits, causal):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
     seed = Nq * 13 + Nk + Hq
     q, k, v = _randn((B, Nq, Hq, D), seed, tdt), _randn((B, Nk, Hkv, D), seed + 1, tdt), _randn((B, Nk, Hkv, D), seed + 2, tdt)
-    n, _ = fa.splitkv_plan(B, Nq, Nk, Hq, D, splits)
+    n, _ = fa.splitkv_plan(B, Nq, Nk, Hq, D, splits, Hkv=Hkv)
     assert n > 1  # these shapes are meant to split
     o, lse = fa.fwd_splitkv(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, num_splits=splits)
     assert fa.status_sync() == fa.FA_OK

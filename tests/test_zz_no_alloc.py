@@ -44,7 +44,7 @@ def _noalloc_abi(q, k, v, o, lse, causal, num_splits=0):
 def test_noalloc_matches_workspace_entry_point_twice(causal):
     for call, seed in enumerate((101, 202)):  # two calls in a row: the scratch keeps the previous contents
         q, k, v = _inputs(seed)
-        n, need = fa.splitkv_plan(q.shape[0], q.shape[1], k.shape[1], q.shape[2], q.shape[3])
+        n, need = fa.splitkv_plan(q.shape[0], q.shape[1], k.shape[1], q.shape[2], q.shape[3], Hkv=k.shape[2])
         assert n > 1 and 0 < need <= fa.NOALLOC_SCRATCH_BYTES
         o_ref, lse_ref = fa.fwd_splitkv(q, k, v, causal=causal)
         o = torch.full_like(q, float("nan"))
