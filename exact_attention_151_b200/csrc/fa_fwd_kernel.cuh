@@ -582,10 +582,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;
     float l_sum = 0.f;
     bool ok = true;
+    // packed heads: a warp whose 32 rows are all past the G Nq real ones only
+    // keeps the hand-offs (its rows' O is never stored)
+    const bool warp_idle = pg && quarter * 32 >= pg * nq;
     for (int j = 0; j <= last; ++j) {
       ok = warp_wait_bar(bar(C::kBarSFull + wg), static_cast<uint32_t>(j & 1), wc);
       if (!ok) break;
       tc_fence_after();
+      if (warp_idle) {
+        tc_fence_before();
+        mbar_arrive(bar(C::kBarPFull + 2 * wg));
+        mbar_arrive(bar(C::kBarPFull + 2 * wg + 1));
+        continue;
+      }
       float s[kTile];
       {
         uint32_t r[4][32];
