@@ -124,7 +124,8 @@ struct Shape {
 };
 
 template <int D, bool FP16>
-fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, float* lse,
+fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                 void* o, float* lse,
                  const Shape& sh, float scale, int causal, cudaStream_t stream, uint64_t limit_ns, int withhold) {
   using C = Cfg<D>;
   auto kernel = fa_fwd_kernel<D, FP16>;
@@ -187,7 +188,7 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.part_o = sh.part_o;
   prm.part_lse = sh.part_lse;
   const int64_t grid = static_cast<int64_t>(prm.n_blocks) * prm.BH * sh.n_splits;
-  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("kernel launch", e);
@@ -294,23 +295,23 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   const void* vb = sh.total_k > 0 ? v : q;
   const int64_t krows = sh.total_k > 0 ? sh.total_k : 1;
   const int64_t khead = sh.total_k > 0 ? sh.Hkv : 1;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   Shape shp = sh;
   shp.pack_g = sh.cu_q == nullptr ? static_cast<int>(pack_group(sh.Nq, sh.Hq, sh.Hkv)) : 0;
   const fa_status mq = shp.pack_g ? make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16, static_cast<uint32_t>(shp.pack_g),
                                               static_cast<uint32_t>(sh.Nq))
                                   : make_tmap(&tq, q, sh.total_q, sh.Hq, sh.D, fp16);
   if (mq != FA_OK || make_tmap(&tk, kb, krows, khead, sh.D, fp16) != FA_OK ||
-      make_tmap(&tv, vb, krows, khead, sh.D, fp16) != FA_OK)
+      make_tmap(&tv, vb, krows, khead, sh.D, fp16) != FA_OK || make_tmap(&to, o, sh.total_q, sh.Hq, sh.D, fp16) != FA_OK)
     return FA_ERR_CUDA;
   if (limit_ns == 0) limit_ns = kDefaultWaitLimitNs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (sh.D == 128) {
-    return fp16 ? launch<128, true>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold)
-                : launch<128, false>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold);
+    return fp16 ? launch<128, true>(dev, tq, tk, tv, to, o, lse, shp, scale, causal, s, limit_ns, withhold)
+                : launch<128, false>(dev, tq, tk, tv, to, o, lse, shp, scale, causal, s, limit_ns, withhold);
   }
-  return fp16 ? launch<64, true>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold)
-              : launch<64, false>(dev, tq, tk, tv, o, lse, shp, scale, causal, s, limit_ns, withhold);
+  return fp16 ? launch<64, true>(dev, tq, tk, tv, to, o, lse, shp, scale, causal, s, limit_ns, withhold)
+              : launch<64, false>(dev, tq, tk, tv, to, o, lse, shp, scale, causal, s, limit_ns, withhold);
 }
 
 Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D) {

@@ -93,7 +93,8 @@ struct Cfg {
   static constexpr int kBarSFull = kBarVEmpty + kVStages;  // [2]: S_i ready
   static constexpr int kBarPFull = kBarSFull + 2;          // [2][2]: half h of P_i written (128 arrivals)
   static constexpr int kBarOFinal = kBarPFull + 4;         // [2]: last PV_i done (single phase)
-  static constexpr int kBarDrain = kBarOFinal + 2;
+  static constexpr int kBarOStaged = kBarOFinal + 2;       // [2]: O_i staged in shared memory (128 arrivals)
+  static constexpr int kBarDrain = kBarOStaged + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024 B
@@ -274,7 +275,8 @@ struct Params {
 template <int D, bool FP16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const Params prm) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const Params prm) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarPFull + 2 * i), 128);
       mbar_init(bar(C::kBarPFull + 2 * i + 1), 128);
       mbar_init(bar(C::kBarOFinal + i), 1);
+      mbar_init(bar(C::kBarOStaged + i), 128);
     }
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
@@ -694,9 +697,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* lse_at = prm.lse + (prm.cu_q != nullptr
                                      ? static_cast<int64_t>(hq) * prm.total_q + q0 + qi
                                      : (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi);
+      // A full dense tile leaves through one TMA store per 64-column slab,
+      // staged in this warpgroup's Q buffer (free: every S_i has completed,
+      // and OFinal_i has been seen) in the 128B-swizzled layout of the map.
+      const bool tma_out = prm.cu_q == nullptr && !pg && (qt + 1) * kTile <= nq;
       if (last >= 0 && ok) {
         tc_fence_after();
         const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
+        uint8_t* qbuf = smem + C::kQOff + wg * C::kTileBytes;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           uint32_t o[32];
@@ -709,10 +717,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    make_float2(inv_l, inv_l));
             pk[k] = row_has_keys ? pack2<FP16>(v.x, v.y) : 0u;
           }
-          if (row_valid) {
+          if (tma_out) {
+            // columns 32q .. 32q+31: slab q / 2, 16-byte chunks 4 (q % 2) .. of the row, swizzled by row % 8
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int chunk = (q & 1) * 4 + k;
+              *reinterpret_cast<uint4*>(qbuf + (q >> 1) * C::kSlabBytes + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+                  make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            }
+          } else if (row_valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
             for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
+        }
+        if (tma_out) {
+          fence_proxy_async_smem();
+          mbar_arrive(bar(C::kBarOStaged + wg));
+          if (quarter == 0 && lane == 0 && wait_bar(bar(C::kBarOStaged + wg), 0, wc)) {
+            for (int hf = 0; hf < C::kHalves; ++hf)
+              tma_store_3d(&tm_o, smem_u32(qbuf) + hf * C::kSlabBytes, hf * 64, h, q0 + qt * kTile);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging buffer must outlive the copy
           }
         }
         if (row_valid) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
