@@ -33,7 +33,7 @@ void set_error(const char* where, cudaError_t e) {
 
 struct DeviceInfo {
   int checked = 0;  // 0 unknown, 1 ok, -1 unsupported
-  unsigned configured = 0;  // bit per kernel instantiation: smem attribute set
+  unsigned configured = 0;  // bit per kernel instantiation: smem attribute set (layout at each launch)
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -128,8 +128,11 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
                  void* o, float* lse,
                  const Shape& sh, float scale, int causal, cudaStream_t stream, uint64_t limit_ns, int withhold) {
   using C = Cfg<D>;
-  auto kernel = fa_fwd_kernel<D, FP16>;
-  const unsigned bit = 1u << ((D == 128 ? 2 : 0) + (FP16 ? 1 : 0));
+  // packed heads leave the second query tile free: it takes a second key range
+  const bool pair = sh.pack_g && sh.n_splits > 1;
+  auto kernel = pair ? fa_fwd_kernel<D, FP16, true> : fa_fwd_kernel<D, FP16, false>;
+  // configured bits: 0-3 unpaired forward, 4-11 backward, 12-15 paired forward
+  const unsigned bit = 1u << ((pair ? 12 : 0) + (D == 128 ? 2 : 0) + (FP16 ? 1 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(g_devices[dev].configured & bit)) {
@@ -187,7 +190,8 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   prm.split_tiles = sh.split_tiles;
   prm.part_o = sh.part_o;
   prm.part_lse = sh.part_lse;
-  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * prm.BH * sh.n_splits;
+  const int64_t cta_splits = pair ? (sh.n_splits + 1) / 2 : sh.n_splits;
+  const int64_t grid = static_cast<int64_t>(prm.n_blocks) * prm.BH * cta_splits;
   kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -207,9 +211,10 @@ fa_status launch(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     }
   }
   if (debug_enabled()) {
-    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d splits=%d grid=%lld smem=%d\n",
+    std::fprintf(stderr, "[fa] fwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d splits=%d%s grid=%lld smem=%d\n",
                  D, FP16 ? "fp16" : "bf16", (long long)sh.B, (long long)sh.Nq, (long long)sh.Nk, (long long)sh.Hq,
-                 (long long)sh.Hkv, sh.cu_q ? "packed" : "dense", causal, sh.n_splits, (long long)grid, C::kSmemBytes);
+                 (long long)sh.Hkv, sh.cu_q ? "packed" : "dense", causal, sh.n_splits, pair ? " paired" : "",
+                 (long long)grid, C::kSmemBytes);
   }
   return FA_OK;
 }
@@ -235,15 +240,17 @@ int64_t pack_group(int64_t Nq, int64_t Hq, int64_t Hkv) {
 }
 
 // Number of key ranges: when the query side alone fills less than half the
-// SMs, as many ranges as keep the CTAs within one wave (one CTA per SM), never
-// more than the key tiles or kMaxSplits; the count is then evened so every
-// range has the same number of tiles.
+// SMs, as many ranges as keep the CTAs within one wave (one CTA per SM; with
+// packed heads a CTA takes two ranges, one per query tile), never more than the
+// key tiles or kMaxSplits; the count is then evened so every range has the same
+// number of tiles.
 int resolve_splits(int requested, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int sm_count,
                    int* tiles_out) {
   const int64_t n_kt = (Nk + kTile - 1) / kTile;
-  const int64_t base = pack_group(Nq, Hq, Hkv) ? B * Hkv : ((Nq + kBlockRows - 1) / kBlockRows) * B * Hq;
+  const bool packed = pack_group(Nq, Hq, Hkv) != 0;
+  const int64_t base = packed ? B * Hkv : ((Nq + kBlockRows - 1) / kBlockRows) * B * Hq;
   int64_t want = requested;
-  if (want <= 0) want = (base >= sm_count / 2 || n_kt < 2) ? 1 : sm_count / base;
+  if (want <= 0) want = (base >= sm_count / 2 || n_kt < 2) ? 1 : (packed ? 2 : 1) * (sm_count / base);
   want = std::max<int64_t>(1, std::min<int64_t>({want, n_kt > 0 ? n_kt : 1, kMaxSplits}));
   const int64_t tiles = (n_kt + want - 1) / want;
   const int64_t splits = tiles > 0 ? (n_kt + tiles - 1) / tiles : 1;

@@ -253,7 +253,7 @@ struct Params {
   int n_blocks;         // ceil(max_nq / 256)
   float scale_log2;
   int causal;           // key j visible to query i iff j <= i + nk - nq (bottom-right aligned)
-  // Split-KV (n_splits > 1, dense shapes only): CTA split s covers key tiles
+  // Split-KV (n_splits > 1, dense shapes only): key range s covers key tiles
   // [s * split_tiles, (s + 1) * split_tiles) and writes its own normalised O
   // and LSE, in fp32, to part_o [n_splits, B, Hq, Nq, D] and part_lse
   // [n_splits, B, Hq, Nq]; a separate kernel merges the splits.
@@ -272,7 +272,13 @@ struct Params {
   int BHq;
 };
 
-template <int D, bool FP16>
+// PAIR (paired split-KV, for packed heads with n_splits > 1): the second query
+// tile holds the same packed queries as the first, and CTA split c computes the
+// partial results of key ranges 2c (tile 0) and 2c + 1 (tile 1) side by side,
+// each tile with its own K and V tiles. A template parameter, so that the
+// unpaired MMA issue loop carries none of its bookkeeping (each instruction of
+// the issuing warp is tensor-pipe time).
+template <int D, bool FP16, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -351,7 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int delta = nk - nq;  // causal offset: query i sees keys j <= i + delta
   const int qt0 = 2 * mb;
   const int qt1 = 2 * mb + 1;
-  const bool q1_valid = !pg && qt1 < n_qt;
+  constexpr bool pair = PAIR;
+  // partial-result slot (split-KV) of tile 0; tile 1 takes the next one when paired
+  const int slot0 = pair ? 2 * split : split;
+  const bool q1_valid = pair ? slot0 + 1 < prm.n_splits : (!pg && qt1 < n_qt);
   // smallest and largest query index held by query tile qt (packed heads:
   // the first and the last query)
   auto q_min = [&](int qt) -> int { return pg ? 0 : qt * kTile; };
@@ -364,18 +373,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (last_key < 0) return -1;
     return min(n_kt - 1, last_key / kTile);
   };
-  // This CTA's key tiles: jb .. je-1 (all of them unless split-KV). Tile
-  // indices below are relative to jb; lastI is the last tile (relative) with a
-  // key visible to some row of query tile I, -1 if none.
-  const int jb = split * prm.split_tiles;
-  const int je = prm.n_splits > 1 ? min(n_kt, jb + prm.split_tiles) : n_kt;
-  auto last_rel = [&](int qt) -> int {
+  // Key tiles of query tile i: jb_i .. je_i - 1 (all of them unless split-KV;
+  // one range for both tiles unless paired). Tile indices below are relative to
+  // jb_i; last_i is the last tile (relative) with a key visible to some row of
+  // query tile i, -1 if none.
+  const int jb0 = slot0 * prm.split_tiles;
+  const int jb1 = pair ? jb0 + prm.split_tiles : jb0;
+  auto last_rel = [&](int qt, int jb) -> int {
+    const int je = prm.n_splits > 1 ? min(n_kt, jb + prm.split_tiles) : n_kt;
     const int t = min(last_key_tile(qt), je - 1);
     return t < jb ? -1 : t - jb;
   };
-  const int last0 = last_rel(qt0);
-  const int last1 = q1_valid ? last_rel(qt1) : -1;
+  const int last0 = last_rel(qt0, jb0);
+  const int last1 = q1_valid ? last_rel(pair ? qt0 : qt1, jb1) : -1;
   const int n_kv = (last1 > last0 ? last1 : last0) + 1;
+  // K and V tiles go through their rings as items, in load order. Unpaired,
+  // item j is key tile jb + j, shared by both query tiles. Paired (last1 <=
+  // last0 there: tile 1's range starts later), items alternate tile 0 and tile 1
+  // while both have tiles, then tile 0's remaining ones follow.
+  const int n_items = pair ? (last0 + 1) + (last1 + 1) : n_kv;
+  auto item_of = [&](int i, int j) -> int { return !pair ? j : (j <= last1 ? 2 * j + i : last1 + 1 + j); };
+  auto item_key_tile = [&](int u) -> int {  // absolute key tile of item u
+    if (!pair) return jb0 + u;
+    if (u < 2 * (last1 + 1)) return ((u & 1) ? jb1 : jb0) + (u >> 1);
+    return jb0 + (u - (last1 + 1));
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarQ), 1);
@@ -413,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loader
     // The whole warp runs this loop (converged); one elected lane issues each
-    // barrier arm and TMA copy.
+    // barrier arm and TMA copy. (A second loader warp for V measured slower: one
+    // more polling warp shares a sub-partition with two softmax warps.)
     {
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -423,48 +446,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (pg) {
         // packed heads: one (64, G, Nq) box per slab fills rows 0 .. G Nq - 1
-        mbar_arrive_expect_tx_elect(bar(C::kBarQ), C::kHalves * pg * nq * 128);
-        for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d_elect(q_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0, bar(C::kBarQ));
+        // (into both query tiles when paired)
+        const int nt = pair ? 2 : 1;
+        mbar_arrive_expect_tx_elect(bar(C::kBarQ), nt * C::kHalves * pg * nq * 128);
+        for (int i = 0; i < nt; ++i)
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_3d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0, bar(C::kBarQ));
       } else {
         mbar_arrive_expect_tx_elect(bar(C::kBarQ), (q1_valid ? 2 : 1) * C::kTileBytes);
         for (int i = 0; i < (q1_valid ? 2 : 1); ++i)
           for (int hf = 0; hf < C::kHalves; ++hf)
             tma_load_3d_elect(q_smem(i) + hf * C::kSlabBytes, &tm_q, hf * 64, h, q0 + (qt0 + i) * kTile, bar(C::kBarQ));
       }
-      const bool withhold = prm.withhold_v_load && blockIdx.x == 0;
-      int nk = 0, nv = 0;  // K and V tiles issued
-      for (int j = 0; j < n_kv; ++j) {
-        const int sk = j % C::kKStages;
-        if (j >= C::kKStages &&
-            !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((j / C::kKStages) & 1) ^ 1), wc))
+      const bool withhold = prm.withhold_v_load && blockIdx.x == 0;  // V item 0 of CTA 0
+      int nk_issued = 0, nv_issued = 0;  // K and V items handled
+      for (int u = 0; u < n_items; ++u) {
+        const int key_row = k0 + item_key_tile(u) * kTile;
+        const int sk = u % C::kKStages;
+        if (u >= C::kKStages &&
+            !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((u / C::kKStages) & 1) ^ 1), wc))
           break;
         mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, k0 + (jb + j) * kTile, bar(C::kBarKFull + sk));
-        nk = j + 1;
-        const int sv = j % C::kVStages;
-        if (j >= C::kVStages &&
-            !warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((j / C::kVStages) & 1) ^ 1), wc))
+          tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, key_row, bar(C::kBarKFull + sk));
+        nk_issued = u + 1;
+        const int sv = u % C::kVStages;
+        if (u >= C::kVStages &&
+            !warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((u / C::kVStages) & 1) ^ 1), wc))
           break;
-        if (!(withhold && j == 0)) {
+        if (!(withhold && u == 0)) {
           mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
           for (int hf = 0; hf < C::kHalves; ++hf)
-            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, k0 + (jb + j) * kTile, bar(C::kBarVFull + sv));
+            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, key_row, bar(C::kBarVFull + sv));
         }
-        nv = j + 1;
+        nv_issued = u + 1;
       }
       // Let every load this thread issued land before shared memory is
       // released (immediate in a normal run, where all were consumed): for
       // each stage, wait for the phase of its last arming.
       drain_wait(bar(C::kBarQ), 0);
-      for (int s = 0; s < C::kKStages && s < nk; ++s) {
-        const int jl = s + ((nk - 1 - s) / C::kKStages) * C::kKStages;
-        drain_wait(bar(C::kBarKFull + s), static_cast<uint32_t>((jl / C::kKStages) & 1));
+      for (int st = 0; st < C::kKStages && st < nk_issued; ++st) {
+        const int ul = st + ((nk_issued - 1 - st) / C::kKStages) * C::kKStages;
+        drain_wait(bar(C::kBarKFull + st), static_cast<uint32_t>((ul / C::kKStages) & 1));
       }
-      for (int s = 0; s < C::kVStages && s < nv; ++s) {
-        const int jl = s + ((nv - 1 - s) / C::kVStages) * C::kVStages;
-        if (!(withhold && jl == 0)) drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((jl / C::kVStages) & 1));
+      for (int st = 0; st < C::kVStages && st < nv_issued; ++st) {
+        const int ul = st + ((nv_issued - 1 - st) / C::kVStages) * C::kVStages;
+        if (!(withhold && ul == 0)) drain_wait(bar(C::kBarVFull + st), static_cast<uint32_t>((ul / C::kVStages) & 1));
       }
     }
     __syncwarp();
@@ -515,10 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      // Both halves of PV_i(j): each waits for its half of P.
-      auto issue_pv = [&](int i, int j, int sv, bool split) -> bool {
+      // Both halves of PV_i(j) with the V item u: each waits for its half of P.
+      auto issue_pv = [&](int i, int j, int u, bool split) -> bool {
+        const int sv = u % C::kVStages;
         if (!warp_wait_bar(bar(C::kBarPFull + 2 * i), static_cast<uint32_t>(j & 1), wc) ||
-            !warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((j / C::kVStages) & 1), wc))
+            !warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((u / C::kVStages) & 1), wc))
           return false;
         tc_fence_after();
         issue_pv_half(i, j, sv, split, 0);
@@ -527,34 +555,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv_half(i, j, sv, split, 1);
         return true;
       };
-      const bool split0 = jb == 0 && split_p_tile(qt0, 0, causal, delta, nk);
-      const bool split1 = jb == 0 && split_p_tile(qt1, 0, causal, delta, nk);
+      const bool split0 = jb0 == 0 && split_p_tile(qt0, 0, causal, delta, nk);
+      const bool split1 = jb1 == 0 && split_p_tile(pair ? qt0 : qt1, 0, causal, delta, nk);
+      // wait for K item u; false if the CTA is aborting
+      auto wait_k = [&](int u) -> bool {
+        if (!warp_wait_bar(bar(C::kBarKFull + u % C::kKStages), static_cast<uint32_t>((u / C::kKStages) & 1), wc))
+          return false;
+        tc_fence_after();
+        return true;
+      };
       bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
       for (int j = 0; ok && j <= n_kv; ++j) {
-        const int sk = j % C::kKStages;
-        if (j < n_kv) {
-          ok = warp_wait_bar(bar(C::kBarKFull + sk), static_cast<uint32_t>((j / C::kKStages) & 1), wc);
-          if (!ok) break;
-          tc_fence_after();
-          if (j <= last0) issue_s(0, sk);
+        if (j < n_kv && (j <= last0 || !pair)) {
+          // S0(j); unpaired, K item j also serves S1(j) and is waited for here
+          const int u = item_of(0, j);
+          if (!(ok = wait_k(u))) break;
+          if (j <= last0) issue_s(0, u % C::kKStages);
+          if (pair && u + C::kKStages < n_items) mma_commit_elect(bar(C::kBarKEmpty + u % C::kKStages));
         }
         if (j >= 1 && j - 1 <= last1) {
           // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
-          const int jp = j - 1, sv = jp % C::kVStages;
-          ok = issue_pv(1, jp, sv, split1 && jp == 0);
+          const int jp = j - 1, u = item_of(1, jp);
+          ok = issue_pv(1, jp, u, split1 && jp == 0);
           if (!ok) break;
           if (jp == last1) mma_commit_elect(bar(C::kBarOFinal + 1));
-          if (jp + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));  // V_jp: last reader done
+          // unpaired: PV1 is V_jp's last reader; paired: its only one
+          if (u + C::kVStages < n_items) mma_commit_elect(bar(C::kBarVEmpty + u % C::kVStages));
         }
         if (j < n_kv) {
-          if (j <= last1) issue_s(1, sk);
-          if (j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + sk));  // K_j: last reader issued
+          if (j <= last1) {
+            const int u = item_of(1, j);
+            if (pair && !(ok = wait_k(u))) break;
+            issue_s(1, u % C::kKStages);
+            if (pair && u + C::kKStages < n_items) mma_commit_elect(bar(C::kBarKEmpty + u % C::kKStages));
+          }
+          // unpaired: K_j's last reader has been issued
+          if (!pair && j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + j % C::kKStages));
           if (j <= last0) {
-            const int sv = j % C::kVStages;
-            ok = issue_pv(0, j, sv, split0 && j == 0);
+            const int u = item_of(0, j);
+            ok = issue_pv(0, j, u, split0 && j == 0);
             if (!ok) break;
             if (j == last0) mma_commit_elect(bar(C::kBarOFinal + 0));
-            if (j > last1 && j + C::kVStages < n_kv) mma_commit_elect(bar(C::kBarVEmpty + sv));
+            if ((pair || j > last1) && u + C::kVStages < n_items) mma_commit_elect(bar(C::kBarVEmpty + u % C::kVStages));
           }
         }
       }
@@ -569,8 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_increase<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = warp / 4;              // query tile of this warpgroup
-    const int qt = qt0 + wg;
+    const int qt = pair ? qt0 : qt0 + wg;  // paired: both tiles hold the same queries
     const int last = wg == 0 ? last0 : last1;
+    const int jb = wg == 0 ? jb0 : jb1;   // first key tile of this tile's range
     const int quarter = warp % 4;         // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     // this row's query index and head (packed heads: row = n G + g)
@@ -661,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_has_keys = row_last_key >= 0 && (!splitkv || row_last_key >= jb * kTile);
     if (splitkv) {
       // fp32 partial result of this key range (normalised by its own sum)
-      const int64_t prow = (static_cast<int64_t>(split) * prm.BHq + static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi;
+      const int64_t prow = (static_cast<int64_t>(slot0 + (pair ? wg : 0)) * prm.BHq + static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi;
       float* orow = prm.part_o + prow * D;
       if (last >= 0 && ok) {
         tc_fence_after();

@@ -47,6 +47,13 @@ def _check(o, lse, o_ref, lse_ref):
     (1, 300, 2048, 2, 2, 128, "bf16", 3),
     (1, 1, 777, 4, 4, 64, "bf16", 64),
     (1, 4, 129, 2, 1, 128, "bf16", 2),
+    # packed heads pair two key ranges per CTA: an odd count (the last CTA's
+    # second range is empty), a shorter second range, ragged last tiles
+    (1, 1, 3000, 8, 2, 128, "bf16", 5),
+    (1, 2, 1100, 16, 4, 64, "fp16", 3),
+    (1, 1, 300, 4, 1, 128, "bf16", 3),
+    (1, 1, 850, 8, 2, 128, "bf16", 4),
+    (2, 3, 700, 8, 2, 64, "bf16", 0),
 ])
 def test_splitkv_matches_oracle(B, Nq, Nk, Hq, Hkv, D, dtype, splits, causal):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
