@@ -111,3 +111,26 @@ def test_backward_workspace_size():
     size = ctypes.c_size_t(0)
     assert lib.fa_bwd_workspace_size(-1, 5, 5, ctypes.byref(size)) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_bwd_workspace_size(1, 5, 5, None) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,Nq,Nk,Hq,Hkv,D", [
+    (1, 1, 32768, 32, 8, 128), (8, 1, 8192, 32, 8, 128), (1, 1, 4096, 32, 8, 128), (2, 1, 1000, 8, 1, 128),
+    (1, 16, 8192, 8, 2, 128), (3, 2, 777, 16, 4, 64), (1, 64, 20000, 4, 4, 128), (1, 300, 2048, 2, 2, 128),
+])
+def test_splitkv_plan_fits_one_wave(B, Nq, Nk, Hq, Hkv, D):
+    """The automatic plan keeps every key range non-empty and the CTAs within one
+    wave of 148 SMs; with packed heads (Nq * G <= 128, G > 1) a CTA takes two
+    ranges, so the CTA count is half the range count per (batch, K/V head)."""
+    splits, ws = fa.splitkv_plan(B, Nq, Nk, Hq, D, 0, Hkv=Hkv)
+    n_kt = -(-Nk // 128)
+    G = Hq // Hkv
+    packed = G > 1 and Nq * G <= 128
+    assert 1 <= splits <= min(n_kt, 64)
+    tiles = -(-n_kt // splits)
+    assert (splits - 1) * tiles < n_kt  # the last range is not empty
+    if packed:
+        ctas = B * Hkv * (-(-splits // 2) if splits > 1 else 1)
+    else:
+        ctas = B * Hq * (-(-Nq // 256)) * splits
+    assert splits == 1 or ctas <= 148
+    assert (ws > 0) == (splits > 1)
