@@ -595,6 +595,13 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
     size_t need = 0;
     fa_status st = fa_fwd_splitkv_plan(B, Nq, Nk, Hq, Hkv, D, num_splits, &splits, &need);
     if (st != FA_OK) return st;
+    int requested = num_splits;
+    // automatic count: fall back to the largest one whose partial results fit
+    for (int r = splits - 1; num_splits == 0 && r >= 1 && need > fa::kNoAllocScratchBytes; --r) {
+      st = fa_fwd_splitkv_plan(B, Nq, Nk, Hq, Hkv, D, r, &splits, &need);
+      if (st != FA_OK) return st;
+      requested = r;
+    }
     if (need > fa::kNoAllocScratchBytes) {
       std::snprintf(fa::g_last_error, sizeof(fa::g_last_error),
                     "split-KV scratch of %zu bytes needed, the built-in scratch holds %zu bytes", need,
@@ -615,7 +622,7 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
       st = fa::noalloc_scratch_address(dev, &scratch);
       if (st != FA_OK) return st;
       int tiles = 0;
-      fa::resolve_splits(num_splits, B, Nq, Nk, Hq, Hkv, fa::device_sm_count(dev), &tiles);
+      fa::resolve_splits(requested, B, Nq, Nk, Hq, Hkv, fa::device_sm_count(dev), &tiles);
       sh.n_splits = splits;
       sh.split_tiles = tiles;
       sh.part_o = static_cast<float*>(scratch);

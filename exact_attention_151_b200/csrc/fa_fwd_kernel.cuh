@@ -32,6 +32,9 @@
 //                      normalises O_i and writes O and LSE.
 // Because S_i(j) is issued after PV_i(j-1), the completion of S_i(j) implies
 // that PV_i(j-1) has finished, so the O_i rescale needs no extra barrier.
+// With packed heads and split-KV (the PAIR instantiation) both query tiles hold
+// the same packed queries and each works through its own key range, so a CTA
+// produces two partial results and both softmax warpgroups stay busy.
 //
 // Online-softmax bookkeeping (base 2, x = s * scale * log2(e)): m is only
 // raised when a tile's max exceeds it by more than kRescaleThreshold, so

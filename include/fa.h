@@ -159,7 +159,8 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
  * when Nq * (Hq / Hkv) <= 128 and Hq / Hkv > 1 the forward packs the query
  * heads that share a key/value head into one tile (one work item per K/V head
  * instead of one per query head), and the key range count is chosen for that
- * smaller grid.
+ * smaller grid (each CTA then computes two ranges, one per query tile of the
+ * kernel, so the plan returns twice the ranges that fill the SMs).
  */
 fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, int num_splits,
                               int* splits_out, size_t* workspace_bytes);
@@ -176,9 +177,11 @@ fa_status fa_fwd_splitkv_plan(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int
  *   provides q, k, v, o and lse.
  *   The partial results go to a scratch buffer compiled into the library:
  *   FA_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every GPU which
- *   loads the library holds until the process exits. Sizes whose partial
+ *   loads the library holds until the process exits. With num_splits = 0 the
+ *   call uses the plan's range count, or the largest smaller count whose
+ *   partial results fit the scratch; an explicit num_splits whose partial
  *   results would not fit (fa_fwd_splitkv_plan's workspace_bytes above that)
- *   return FA_ERR_UNSUPPORTED without launching, with the sizes in
+ *   returns FA_ERR_UNSUPPORTED without launching, with the sizes in
  *   fa_last_error().
  *   No cudaMalloc, cudaFree or other allocating call is made. The first call
  *   on each device looks up the scratch buffer's device address

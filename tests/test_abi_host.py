@@ -134,3 +134,15 @@ def test_splitkv_plan_fits_one_wave(B, Nq, Nk, Hq, Hkv, D):
         ctas = B * Hq * (-(-Nq // 256)) * splits
     assert splits == 1 or ctas <= 148
     assert (ws > 0) == (splits > 1)
+
+
+def test_noalloc_scratch_has_a_fitting_range_count():
+    """Packed heads double the automatic range count, so some plans outgrow the
+    no-allocation scratch; fa_fwd_splitkv_noalloc then falls back to the largest
+    smaller count that fits, which always exists (one range needs none)."""
+    scratch = 16 << 20
+    B, Nq, Nk, Hq, Hkv, D = 1, 16, 65536, 32, 4, 128
+    splits, need = fa.splitkv_plan(B, Nq, Nk, Hq, D, 0, Hkv=Hkv)
+    assert need > scratch
+    fits = [r for r in range(splits - 1, 0, -1) if fa.splitkv_plan(B, Nq, Nk, Hq, D, r, Hkv=Hkv)[1] <= scratch]
+    assert fits and fa.splitkv_plan(B, Nq, Nk, Hq, D, fits[0], Hkv=Hkv)[0] > 1
