@@ -17,9 +17,9 @@
 //   * causal attention skips future positions: handbook ch. 3, practical notes.
 //
 // Blackwell mapping (prior art on the pages targets Ampere; this is not it):
-//   warp 9 (loader)    TMA 4-D tiled loads: Q0 and Q1 once, K_j and V_j into
+//   warp 9 (loader)    TMA 3-D tiled loads: Q0 and Q1 once, K_j and V_j into
 //                      separate rings of 128B-swizzled shared-memory tiles;
-//   warp 8 (MMA)       one thread issues tcgen05.mma in the order
+//   warp 8 (MMA)       an elected lane of the converged warp issues tcgen05.mma in the order
 //                        S0(j), PV1(j-1), S1(j), PV0(j)
 //                      so that while one softmax warpgroup works on its
 //                      scores the tensor cores serve the other query tile;
