@@ -2,19 +2,22 @@
 """Benchmark of the fused exact-attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--pass fwd|bwd]
+                    [--pass fwd|bwd] [--shard]
 
-One step = one fa_fwd call over the whole workload (default: the Llama-7B-shaped
-causal forward, B=4 H=32 N=2048 D=128 bf16). Prints ONE JSON line on rank 0.
+One step = one fa_fwd call over the whole workload (default: the sequence-sweep
+point N=32768, B=1 H=16 D=128 bf16 non-causal, the largest single-GPU
+configuration and inside the "non-causal, N >= 4k" range the forward's target
+is stated on). Prints ONE JSON line on rank 0.
 
   value      forward TFLOP/s of the whole job (4*B*H*N^2*D per step, halved for
              causal) with inputs resident in HBM; device time from CUDA events
              around exactly K steps (barrier + synchronize on both sides), max
-             over ranks. Q+K+V+O (256 MiB at the default) exceed the 126 MB L2,
+             over ranks. Q+K+V+O (512 MiB at the default) exceed the 126 MB L2,
              so no flush is done between steps.
   e2e        the same metric through the public API with pinned host buffers:
              each step copies Q, K, V host->device, runs fa_fwd and copies O and
-             LSE back, all inside the timed region.
+             LSE back, all inside the timed region; two buffer sets and three
+             streams let the copies of neighbouring steps overlap the kernels.
   roofline   tensor-core bound: achieved TFLOP/s of the kernel against the
              measured cuBLAS bf16 peak; dram traffic per launch from the
              committed ncu summary when it matches the current kernel source.
@@ -27,8 +30,12 @@ flops (five N x N x D products against the forward's two); its e2e copies q,
 k, v, o, lse and dO in and dQ, dK, dV out, and its cpu_baseline is the oracle's
 backward on one (batch, head) slice.
 
-With torchrun (N>1) every rank runs the full workload on its own GPU (weak
-scaling, no collective on the data path); the timing is reduced with MAX.
+With torchrun (N>1) every rank runs the full workload on its own GPU by
+default (weak scaling: the job is N independent copies of the workload, no
+collective on the data path); the timing is reduced with MAX. --shard splits
+ONE workload over the ranks instead (contiguous batch slices, or head slices
+when B < N) and ends every step with an NCCL all-gather of O and LSE, so each
+rank holds the whole result (strong scaling).
 """
 
 from __future__ import annotations
@@ -48,7 +55,7 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
 METRIC_BWD = "attention bwd TFLOPS (bf16, d=128) and % of B200 dense tensor peak"
 BWD_FLOP_FACTOR = 2.5  # backward flops per forward flop (5 vs 2 matrix products)
-DEFAULT_WORKLOAD = "llama7b_b4h32n2048d128_causal"
+DEFAULT_WORKLOAD = "sweep_n32768_noncausal"
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_151_b200", "csrc", f) for f in ("fa_fwd.cu", "fa_fwd_kernel.cuh", "sm100.cuh")]
 BWD_KERNEL_SOURCES = KERNEL_SOURCES + [os.path.join(ROOT, "exact_attention_151_b200", "csrc", "fa_bwd_kernel.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -357,36 +364,25 @@ def run_backward(args, w, dev, world, rank):
     value = flops * args.steps * world / (max_ms * 1e-3) / 1e12
     avg_ms = sum(launch_ms) / len(launch_ms)
 
-    # end to end: inputs host->device, backward, gradients device->host
+    # end to end: inputs host->device, backward, gradients device->host (overlapped across steps)
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
-    hosts = [t.pin_memory() for t in (q, k, v, od.cpu(), lsed.cpu(), dout)]
-    devs = [qd, kd, vd, od, lsed, dod]
-    outs_h = [torch.empty_like(q).pin_memory() for _ in range(3)]
+    host_in = [t.pin_memory() for t in (q, k, v, od.cpu(), lsed.cpu(), dout)]
+    slot0 = {"inputs": [qd, kd, vd, od, lsed, dod], "outputs": [dq, dk, dv]}
+    slot1 = {"inputs": [t.clone() for t in slot0["inputs"]], "outputs": [torch.empty_like(t) for t in (dq, dk, dv)]}
+    slots = [slot0, slot1]
+    for sl in slots:
+        sl["host_out"] = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sl["outputs"]]
 
-    def e2e_step():
-        for d_, h_ in zip(devs, hosts):
-            d_.copy_(h_, non_blocking=True)
-        step()
-        for h_, d_ in zip(outs_h, (dq, dk, dv)):
-            h_.copy_(d_, non_blocking=True)
+    def compute(sl):
+        q_, k_, v_, o_, l_, do_ = sl["inputs"]
+        dq_, dk_, dv_ = sl["outputs"]
+        fa.bwd(q_, k_, v_, o_, l_, do_, scale=w.softmax_scale, causal=w.causal, dq=dq_, dk=dk_, dv=dv_,
+               workspace=workspace)
 
-    e2e_step()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        dist.barrier()
-    e2e_value = flops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
-    h2d = sum(h_.numel() * h_.element_size() for h_ in hosts)
-    d2h = sum(h_.numel() * h_.element_size() for h_ in outs_h)
+    e2e_ms = pipelined_e2e(dev, e2e_steps, host_in, slots, compute, world)
+    h2d = sum(h_.numel() * h_.element_size() for h_ in host_in)
+    d2h = sum(h_.numel() * h_.element_size() for h_ in slot0["host_out"])
+    e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
 
     if rank == 0:
         peak, peak_sus, peak_src = measured_peak()
@@ -406,7 +402,10 @@ def run_backward(args, w, dev, world, rank):
                          "note": "achieved and frac: the whole step (preprocess, dQ and dK/dV kernels); traffic: the "
                                  "dominant dK/dV kernel's DRAM bytes per launch"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                    "pcie_gbs": (h2d + d2h) * e2e_steps / (e2e_ms * 1e-3) / 1e9,
+                    "overlap": "two buffer sets; host->device copies, kernels and device->host copies on three "
+                               "streams"},
             "clocks": clocks.summary(),
             "gpu_launches": args.steps * 3,
             "kernel_source_hash": kernel_source_hash(BWD_KERNEL_SOURCES),
@@ -458,6 +457,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
+    ap.add_argument("--shard", action="store_true",
+                    help="split one workload over the ranks (batch or heads) and all-gather O and LSE each step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -493,25 +494,128 @@ def main():
     if args.which == "bwd":
         return run_backward(args, w, dev, world, rank)
 
+    return run_forward(args, w, dev, world, rank)
+
+
+def pipelined_e2e(dev, n_steps, host_in, slots, compute, world):
+    """End-to-end time of n_steps steps through the public API, in ms (max over ranks).
+
+    Every step copies its inputs host->device from pinned buffers (``host_in``),
+    runs ``compute(slot)`` and copies the slot's results device->host. Two
+    buffer sets (``slots``: dicts with device "inputs", device "outputs" and
+    pinned "host_out") alternate, and the copies in, the kernels and the copies
+    out run on three streams, so the input copy of step i+1 and the output copy
+    of step i-1 overlap the kernels of step i. A slot's inputs are only
+    overwritten after the kernels of two steps back have read them, and its
+    outputs only after they have been copied out."""
+    import torch
+    import torch.distributed as dist
+
+    comp, up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d = [torch.cuda.Event() for _ in slots]
+    done = [torch.cuda.Event() for _ in slots]
+    d2h = [torch.cuda.Event() for _ in slots]
+
+    def one(i):
+        s = i % len(slots)
+        sl = slots[s]
+        up.wait_event(done[s])
+        with torch.cuda.stream(up):
+            for d_, h_ in zip(sl["inputs"], host_in):
+                d_.copy_(h_, non_blocking=True)
+        h2d[s].record(up)
+        comp.wait_event(h2d[s])
+        comp.wait_event(d2h[s])
+        with torch.cuda.stream(comp):
+            compute(sl)
+        done[s].record(comp)
+        down.wait_event(done[s])
+        with torch.cuda.stream(down):
+            for h_, d_ in zip(sl["host_out"], sl["outputs"]):
+                h_.copy_(d_, non_blocking=True)
+        d2h[s].record(down)
+
+    for i in range(len(slots)):  # warm-up: every event recorded once
+        one(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    up.wait_event(e0)
+    down.wait_event(e0)
+    for i in range(n_steps):
+        one(i)
+    for ev in d2h:
+        comp.wait_event(ev)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    return float(te.item())
+
+
+def run_forward(args, w, dev, world, rank):
+    """Time fa_fwd (or the split-KV pair of kernels) over the workload; with --shard, one workload split
+    over the ranks plus the all-gather of O and LSE."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_151_b200 as fa
+    from exact_attention_151_b200.inputs import make_qkv
+    from exact_attention_151_b200.sharding import ForwardSharding
+
     q, k, v = make_qkv(w)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    od = torch.empty_like(qd)
-    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    shard = None
+    if args.shard:
+        if not is_square(w) or w.splitkv:
+            raise SystemExit("--shard needs a square self-attention workload")
+        shard = [ForwardSharding(w.B, w.N, w.H, w.D, world, rank, dev, q.dtype) for _ in range(2)]
+        q_in, k_in, v_in = (shard[0].local(t) for t in (q, k, v))
+    else:
+        q_in, k_in, v_in = q, k, v
+    lse_shape = shard[0].local_lse_shape() if shard else (w.B, w.H, w.N)
+
+    def make_slot():
+        qd_, kd_, vd_ = q_in.to(dev), k_in.to(dev), v_in.to(dev)
+        return {"inputs": [qd_, kd_, vd_],
+                "o": torch.empty_like(qd_), "lse": torch.empty(lse_shape, dtype=torch.float32, device=dev)}
+
+    slots = [make_slot(), make_slot()]
     flush = None
     if w.min_hbm_bytes <= 126e6:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
     kernels_per_step = 1
+    workspace = None
     if w.splitkv:
         n_splits, ws_bytes = fa.splitkv_plan(w.B, w.N, w.n_keys, w.H, w.D, Hkv=w.kv_heads)
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         kernels_per_step = 2 if n_splits > 1 else 1
 
-    def step():
+    def compute(sl, s_idx=0):
+        qd_, kd_, vd_ = sl["inputs"]
         if w.splitkv:
-            fa.fwd_splitkv(qd, kd, vd, scale=w.softmax_scale, causal=w.causal, workspace=workspace, o=od, lse=lsed)
+            fa.fwd_splitkv(qd_, kd_, vd_, scale=w.softmax_scale, causal=w.causal, workspace=workspace, o=sl["o"],
+                           lse=sl["lse"])
         else:
-            fa.fwd_into(qd, kd, vd, od, lsed, scale=w.softmax_scale, causal=w.causal)
+            fa.fwd_into(qd_, kd_, vd_, sl["o"], sl["lse"], scale=w.softmax_scale, causal=w.causal)
+        if shard:
+            sl["shard"].exchange(sl["o"], sl["lse"])
+
+    if shard:
+        for sl, sh in zip(slots, shard):
+            sl["shard"] = sh
+            sl["outputs"] = [sh.o_recv, sh.l_recv]
+    else:
+        for sl in slots:
+            sl["outputs"] = [sl["o"], sl["lse"]]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        compute(slots[0])
 
     for _ in range(args.warmup):
         step()
@@ -549,50 +653,36 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     max_ms = float(t.item())
     ms_per_step = max_ms / args.steps
-    value = w.flops * args.steps * world / (max_ms * 1e-3) / 1e12
+    # replicas: every rank does the whole workload; --shard: the ranks share one
+    job_flops = w.flops * (1 if shard else world)
+    value = job_flops * args.steps / (max_ms * 1e-3) / 1e12
     avg_launch_ms = sum(launch_ms) / len(launch_ms)
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers, copies overlapped with the kernels
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 50))
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    oh = torch.empty_like(qh).pin_memory()
-    lseh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step()
-        oh.copy_(od, non_blocking=True)
-        lseh.copy_(lsed, non_blocking=True)
-
-    e2e_step()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        dist.barrier()
-    e2e_value = w.flops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
-    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
-    d2h = q.numel() * q.element_size() + lseh.numel() * 4
+    host_in = [t.pin_memory() for t in (q_in, k_in, v_in)]
+    for sl in slots:
+        sl["host_out"] = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sl["outputs"]]
+    e2e_ms = pipelined_e2e(dev, e2e_steps, host_in, slots, compute, world)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in slots[0]["host_out"])
+    e2e_value = job_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
 
     if rank == 0:
         peak, peak_sus, peak_src = measured_peak()
-        achieved = w.flops / (avg_launch_ms * 1e-3) / 1e12
+        kernel_flops = w.flops / world if shard else w.flops
+        achieved = kernel_flops / (avg_launch_ms * 1e-3) / 1e12
         traffic, traffic_how = recorded_traffic(w.name)
         intensity = w.flops / w.min_hbm_bytes
+        cfg = workload_config(w)
+        if shard:
+            cfg["parallelism"] = (f"shard over {'batch' if shard[0].axis == 0 else 'heads'} on {world} rank(s) "
+                                  "+ NCCL all-gather of O and LSE (inside each step)")
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": workload_config(w),
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": ({"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                           "frac": achieved / peak, "traffic": traffic,
@@ -609,7 +699,10 @@ def main():
                           "arithmetic_intensity_flop_per_byte": intensity,
                           "note": "per-step time covers the attention kernel and the split merge kernel"}),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                    "pcie_gbs": (h2d + d2h) * e2e_steps / (e2e_ms * 1e-3) / 1e9,
+                    "overlap": "two buffer sets; host->device copies, kernels and device->host copies on three "
+                               "streams"},
             "clocks": clocks.summary(),
             "gpu_launches": args.steps * kernels_per_step,
             "kernel_source_hash": kernel_source_hash(),
@@ -618,8 +711,12 @@ def main():
             from tests.parity import metrics, passes
 
             rows, o_ref, lse_ref, dt, threads = oracle_row_sample(w, q, k, v, args.cpu_seconds)
-            o_gpu = od.cpu().to(torch.float64).numpy()
-            l_gpu = lsed.cpu().to(torch.float64).numpy()
+            if shard:
+                o_all, l_all = shard[0].assemble()
+            else:
+                o_all, l_all = slots[0]["o"], slots[0]["lse"]
+            o_gpu = o_all.cpu().to(torch.float64).numpy()
+            l_gpu = l_all.cpu().to(torch.float64).numpy()
             m = metrics(o_gpu[rows[:, 0], rows[:, 2], rows[:, 1]], l_gpu[rows[:, 0], rows[:, 1], rows[:, 2]],
                         o_ref, lse_ref)
             line["cpu_baseline"] = {

@@ -18,7 +18,7 @@ import os
 
 __all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "bwd", "bwd_workspace_size", "status_sync", "FaError", "library_path", "load_library",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
-           "FA_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
+           "FA_ERR_TIMEOUT", "FA_ERR_DEVICE_CHECK", "EXPORTED_SYMBOLS", "load_checking_library"]
 
 FA_OK = 0
 FA_ERR_INVALID_ARG = 1
@@ -26,6 +26,7 @@ FA_ERR_UNSUPPORTED = 2
 FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
+FA_ERR_DEVICE_CHECK = 6
 
 FA_BF16 = 0
 FA_FP16 = 1
@@ -37,7 +38,9 @@ EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa",
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
+_CHECKS_LIB_FILE = os.path.join(_HERE, "libfa_b200_checks.so")
 _lib = None
+_checks_lib = None
 
 
 class FaError(RuntimeError):
@@ -56,12 +59,25 @@ def library_path() -> str:
 def load_library():
     """Load the in-tree CUDA library (raises if it has not been built)."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(_LIB_FILE):
-        raise RuntimeError(f"CUDA library {_LIB_FILE} is missing; build it with "
+    if _lib is None:
+        _lib = _open(_LIB_FILE)
+    return _lib
+
+
+def load_checking_library():
+    """Load the checking build (libfa_b200_checks.so: device-side index checks
+    before every global store, reported as FA_ERR_DEVICE_CHECK); same C ABI."""
+    global _checks_lib
+    if _checks_lib is None:
+        _checks_lib = _open(_CHECKS_LIB_FILE)
+    return _checks_lib
+
+
+def _open(path):
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing; build it with "
                            "`python -m exact_attention_151_b200.build`")
-    lib = ctypes.CDLL(_LIB_FILE)
+    lib = ctypes.CDLL(path)
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.fa_status_string.argtypes = [i32]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -93,7 +109,6 @@ def load_library():
     lib.fa_bwd.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
-    _lib = lib
     return lib
 
 

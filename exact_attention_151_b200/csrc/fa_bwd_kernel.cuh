@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       // warpgroup 0 writes dK (scaled), warpgroup 1 dV
-      const bool row_valid = r_abs < N;
+      const bool row_valid = r_abs < N && index_ok(static_cast<int64_t>(b) * prm.H + h < prm.BH && h < prm.H);
       uint16_t* dst_row = (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
       const float mul = wg == 1 ? 1.f : prm.scale;
       constexpr int kCols = D;
@@ -771,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       // warpgroup h writes dQ columns h D/2 .. (scaled)
-      const bool row_valid = r_abs < N;
+      const bool row_valid = r_abs < N && index_ok(static_cast<int64_t>(b) * prm.H + h < prm.BH && h < prm.H);
       uint16_t* dst_row = prm.out0 + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D + wg * (D / 2);
       const uint32_t acc = tmem + lane_base + C::kColAcc + wg * (D / 2);
 #pragma unroll

@@ -41,10 +41,15 @@ std::mutex g_mutex;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// FA_DEBUG, or the pages' names for their library's debug switch
+// (FLASH_ATTN_DEBUG, FLASH_ATTENTION_DEBUG), read once.
 bool debug_enabled() {
   static const bool on = [] {
-    const char* e = std::getenv("FA_DEBUG");
-    return e && *e && *e != '0';
+    for (const char* name : {"FA_DEBUG", "FLASH_ATTN_DEBUG", "FLASH_ATTENTION_DEBUG"}) {
+      const char* e = std::getenv(name);
+      if (e && *e && *e != '0') return true;
+    }
+    return false;
   }();
   return on;
 }
@@ -485,6 +490,39 @@ fa_status noalloc_scratch_address(int dev, void** out) {
   return FA_OK;
 }
 
+// Synchronise `s`, then read and clear the status word (fa_status_sync).
+fa_status sync_status(cudaStream_t s) {
+  unsigned int word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    set_error("cudaStreamSynchronize", cudaGetLastError());
+    return FA_ERR_CUDA;
+  }
+  if (cudaMemcpyFromSymbolAsync(&word, g_status_word, sizeof(word), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    set_error("reading the status word", cudaGetLastError());
+    return FA_ERR_CUDA;
+  }
+  if (word == 0) return FA_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_status_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    set_error("clearing the status word", cudaGetLastError());
+    return FA_ERR_CUDA;
+  }
+  if (word & 1u) return FA_ERR_TIMEOUT;
+  if (word & 2u) return FA_ERR_INVALID_ARG;
+  return FA_ERR_DEVICE_CHECK;
+}
+
+// Common exit of the entry points: with the debug switch on, a call that
+// enqueued work waits for it and returns the device-side status itself.
+fa_status finish(fa_status st, fa_stream_t stream, const char* what) {
+  if (st != FA_OK || !debug_enabled()) return st;
+  const fa_status dev = sync_status(reinterpret_cast<cudaStream_t>(stream));
+  if (dev != FA_OK) std::fprintf(stderr, "[fa] %s: device status %d after the call\n", what, static_cast<int>(dev));
+  return dev;
+}
+
 }  // namespace fa
 
 extern "C" {
@@ -499,6 +537,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: a base pointer is not 16-byte aligned";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA runtime call failed";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait ran out; outputs are invalid";
+    case FA_ERR_DEVICE_CHECK: return "FA_ERR_DEVICE_CHECK: a device-side index check failed; outputs are invalid";
   }
   return "FA_ERR_UNKNOWN";
 }
@@ -506,7 +545,8 @@ const char* fa_status_string(fa_status s) {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N, int64_t H,
                  int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
   try {
-    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream, 0, 0);
+    return fa::finish(fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream, 0, 0),
+                      stream, "fa_fwd");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -516,7 +556,9 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
                      int64_t Nk, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal, fa_dtype dtype,
                      fa_stream_t stream) {
   try {
-    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, Nq, Nk, Hq, Hkv, D), scale, causal, dtype, stream, 0, 0);
+    return fa::finish(
+        fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, Nq, Nk, Hq, Hkv, D), scale, causal, dtype, stream, 0, 0), stream,
+        "fa_fwd_gqa");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -529,7 +571,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   try {
     if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
     fa::Shape sh{cu_seqlens_q, cu_seqlens_k, B, 0, 0, total_q, total_k, max_seqlen_q, Hq, Hkv, D};
-    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
+    return fa::finish(fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0), stream, "fa_fwd_varlen");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -580,7 +622,7 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
       sh.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                              fa::align256(static_cast<size_t>(splits * B * Hq * Nq * D) * 4));
     }
-    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
+    return fa::finish(fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0), stream, "fa_fwd_splitkv");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -629,7 +671,8 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
       sh.part_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) +
                                              fa::align256(static_cast<size_t>(splits * B * Hq * Nq * D) * 4));
     }
-    return fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0);
+    return fa::finish(fa::fwd_impl(q, k, v, o, lse, sh, scale, causal, dtype, stream, 0, 0), stream,
+                      "fa_fwd_splitkv_noalloc");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -639,8 +682,9 @@ fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, flo
                        int64_t H, int64_t D, float scale, int causal, fa_dtype dtype, fa_stream_t stream,
                        uint64_t wait_limit_ns, int withhold_v_load) {
   try {
-    return fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream,
-                        wait_limit_ns, withhold_v_load ? 1 : 0);
+    return fa::finish(fa::fwd_impl(q, k, v, o, lse, fa::dense_shape(B, N, N, H, H, D), scale, causal, dtype, stream,
+                                    wait_limit_ns, withhold_v_load ? 1 : 0),
+                      stream, "fa_fwd_debug");
   } catch (...) {
     return FA_ERR_CUDA;
   }
@@ -656,36 +700,20 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
                  fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
   try {
-    return fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H, D, scale, causal, dtype, workspace,
-                        workspace_bytes, stream);
+    return fa::finish(fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H, D, scale, causal, dtype, workspace,
+                                    workspace_bytes, stream),
+                      stream, "fa_bwd");
   } catch (...) {
     return FA_ERR_CUDA;
   }
 }
 
 fa_status fa_status_sync(fa_stream_t stream) {
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned int word = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess) {
-    cudaGetLastError();
+  try {
+    return fa::sync_status(reinterpret_cast<cudaStream_t>(stream));
+  } catch (...) {
     return FA_ERR_CUDA;
   }
-  if (cudaMemcpyFromSymbolAsync(&word, fa::g_status_word, sizeof(word), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaStreamSynchronize(s) != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_CUDA;
-  }
-  if (word != 0) {
-    const unsigned int zero = 0;
-    const fa_status which = (word & 1u) ? FA_ERR_TIMEOUT : FA_ERR_INVALID_ARG;
-    if (cudaMemcpyToSymbolAsync(fa::g_status_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
-    }
-    return which;
-  }
-  return FA_OK;
 }
 
 }  // extern "C"

@@ -52,9 +52,25 @@ namespace fa {
 
 using namespace sm100;
 
-// Device status word: bit 0 set when some wait ran out. Read and cleared by
-// fa_status_sync. A static __device__ variable, so the library allocates nothing.
+// Device status word: bit 0 set when some wait ran out, bit 1 for packed
+// sequences with inconsistent offsets, bit 2 when a device-side index check of
+// the checking build (FA_CHECKS) failed. Read and cleared by fa_status_sync. A
+// static __device__ variable, so the library allocates nothing.
 __device__ unsigned int g_status_word;
+
+// Checking build (-DFA_CHECKS): every global store is preceded by a check that
+// its index lies inside the tensor the host described; a failed check sets
+// bit 2 of the status word and the store is skipped (no trap). In the normal
+// build the check compiles to `true`.
+__device__ __forceinline__ bool index_ok(bool in_range) {
+#ifdef FA_CHECKS
+  if (!in_range) atomicOr(&g_status_word, 4u);
+  return in_range;
+#else
+  (void)in_range;
+  return true;
+#endif
+}
 
 constexpr int kTile = 128;        // query rows per tile = keys per tile = TMEM lanes
 constexpr int kBlockRows = 256;   // query rows per CTA (two tiles)
@@ -709,6 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // fp32 partial result of this key range (normalised by its own sum)
       const int64_t prow = (static_cast<int64_t>(slot0 + (pair ? wg : 0)) * prm.BHq + static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi;
       float* orow = prm.part_o + prow * D;
+      const bool prow_ok =
+          !row_valid || index_ok(prow >= 0 && prow < static_cast<int64_t>(prm.n_splits) * prm.BHq * prm.Nq);
       if (last >= 0 && ok) {
         tc_fence_after();
         const float inv_l = row_has_keys ? 1.f / l_sum : 0.f;
@@ -717,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_ld32(o_col + q * 32, o);
           tmem_wait_ld();
-          if (row_valid) {
+          if (row_valid && prow_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -731,18 +749,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (row_valid) prm.part_lse[prow] = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
-      } else if (last < 0 && row_valid) {
+        if (row_valid && prow_ok) prm.part_lse[prow] = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+      } else if (last < 0 && row_valid && prow_ok) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
         for (int k = 0; k < D / 4; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
         prm.part_lse[prow] = -INFINITY;
+      } else if (row_valid && prow_ok) {
+        // a wait ran out: mark this range's partial result invalid so the merge
+        // yields NaN rather than combining what an earlier call left behind
+        prm.part_lse[prow] = __int_as_float(0x7fc00000);
       }
     } else {
       uint16_t* orow = prm.out + (static_cast<int64_t>(q0 + qi) * prm.Hq + hq) * D;
-      float* lse_at = prm.lse + (prm.cu_q != nullptr
-                                     ? static_cast<int64_t>(hq) * prm.total_q + q0 + qi
-                                     : (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi);
+      const int64_t lse_idx = prm.cu_q != nullptr ? static_cast<int64_t>(hq) * prm.total_q + q0 + qi
+                                                  : (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Nq + qi;
+      float* lse_at = prm.lse + lse_idx;
+      // dense: lse is [B, Hq, Nq]; packed: [Hq, total_q]
+      const int64_t lse_len = prm.cu_q != nullptr ? static_cast<int64_t>(prm.Hq) * prm.total_q
+                                                  : static_cast<int64_t>(prm.BHq) * prm.Nq;
+      const bool out_ok = !row_valid || index_ok(q0 + qi >= 0 && q0 + qi < prm.total_q && hq >= 0 && hq < prm.Hq &&
+                                                 lse_idx >= 0 && lse_idx < lse_len);
       // A full dense tile leaves through one TMA store per 64-column slab,
       // staged in this warpgroup's Q buffer (free: every S_i has completed,
       // and OFinal_i has been seen) in the 128B-swizzled layout of the map.
@@ -771,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(qbuf + (q >> 1) * C::kSlabBytes + row * 128 + ((chunk ^ (row & 7)) << 4)) =
                   make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
-          } else if (row_valid) {
+          } else if (row_valid && out_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
             for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
@@ -780,15 +807,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tma_out) {
           fence_proxy_async_smem();
           mbar_arrive(bar(C::kBarOStaged + wg));
-          if (quarter == 0 && lane == 0 && wait_bar(bar(C::kBarOStaged + wg), 0, wc)) {
+          if (quarter == 0 && lane == 0 && wait_bar(bar(C::kBarOStaged + wg), 0, wc) &&
+              index_ok(q0 + (qt + 1) * kTile <= prm.total_q && h < prm.Hq)) {
             for (int hf = 0; hf < C::kHalves; ++hf)
               tma_store_3d(&tm_o, smem_u32(qbuf) + hf * C::kSlabBytes, hf * 64, h, q0 + qt * kTile);
             bulk_commit_group();
             bulk_wait_group_read0();  // the staging buffer must outlive the copy
           }
         }
-        if (row_valid) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
-      } else if (last < 0 && row_valid) {
+        if (row_valid && out_ok) *lse_at = row_has_keys ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+      } else if (last < 0 && row_valid && out_ok) {
         // no key tile at all for this query tile
         uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll

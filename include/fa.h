@@ -31,6 +31,22 @@
  * and leave o and lse untouched. A successful return means the work was
  * enqueued on `stream`; device-side timeouts are reported later through
  * fa_status_sync. No C++ exception ever crosses this boundary.
+ *
+ * Debugging (the pages name a debug switch for their library: FLASH_ATTN_DEBUG
+ * on the jsqmd.com page, usage notes; FLASH_ATTENTION_DEBUG on the mlqm.cn
+ * page, section 6.2). With FA_DEBUG (or either of those names) set to a
+ * nonzero value in the environment when the library is first used, every
+ * call prints its launch configuration to stderr and, after enqueueing,
+ * synchronises `stream` and reads the status word itself: a device-side
+ * failure is then returned by the call (FA_ERR_TIMEOUT, FA_ERR_INVALID_ARG,
+ * FA_ERR_DEVICE_CHECK) instead of by a later fa_status_sync. Calls become
+ * synchronous; results are unchanged.
+ *
+ * Checking build: libfa_b200_checks.so is the same library compiled with
+ * -DFA_CHECKS. Before every global-memory store its kernels check that the
+ * index lies inside the output the host described; a failed check skips the
+ * store, sets the status word (FA_ERR_DEVICE_CHECK from fa_status_sync) and
+ * never traps. Results of a passing run are bit-identical to the normal build.
  */
 #ifndef FA_B200_FA_H_
 #define FA_B200_FA_H_
@@ -56,7 +72,8 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, sizes beyond the limits below, or not an sm_100 device */
   FA_ERR_MISALIGNED = 3,  /* a base pointer is not 16-byte aligned */
   FA_ERR_CUDA = 4,        /* a CUDA runtime call failed (no device, launch failure, ...) */
-  FA_ERR_TIMEOUT = 5      /* a device-side wait ran out (reported by fa_status_sync) */
+  FA_ERR_TIMEOUT = 5,     /* a device-side wait ran out (reported by fa_status_sync) */
+  FA_ERR_DEVICE_CHECK = 6 /* checking build only: a device-side index check failed (reported by fa_status_sync) */
 } fa_status;
 
 /* Limits checked before launch: D in {64,128}; B*H*ceil(N/256) <= 2^31-1;
@@ -201,8 +218,10 @@ fa_status fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, vo
  * fa_status_sync - synchronise `stream`, then read and clear this device's
  * status word. Returns FA_OK; FA_ERR_TIMEOUT if a kernel on this device gave
  * up on a bounded wait since the last call (its outputs are then invalid);
- * FA_ERR_INVALID_ARG if fa_fwd_varlen met inconsistent sequence offsets; or
- * FA_ERR_CUDA if the synchronisation itself failed.
+ * FA_ERR_INVALID_ARG if fa_fwd_varlen met inconsistent sequence offsets;
+ * FA_ERR_DEVICE_CHECK if a device-side index check of the checking build
+ * failed; or FA_ERR_CUDA if the synchronisation itself failed. When several
+ * were recorded, the first of that list is returned (all are cleared).
  */
 fa_status fa_status_sync(fa_stream_t stream);
 

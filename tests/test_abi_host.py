@@ -26,8 +26,14 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, s), s
 
 
+def test_checking_build_exports_every_declared_symbol():
+    lib = fa.load_checking_library()
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+
+
 def test_status_strings():
-    for code in range(6):
+    for code in range(7):
         assert fa.status_string(code).startswith("FA_")
     assert "UNKNOWN" in fa.status_string(99)
 
