@@ -112,13 +112,21 @@ double finish_row(const Problem& p, const double* s, int64_t nvis, const std::ve
                   double* o_out) {
   double m = -std::numeric_limits<double>::infinity();
   for (int64_t j = 0; j < nvis; ++j) m = s[j] > m ? s[j] : m;
+  // the unnormalised weights exp(s_j - m), each evaluated once
+  std::vector<double> e(static_cast<size_t>(nvis));
   double l = 0.0;
-  for (int64_t j = 0; j < nvis; ++j) l += std::exp(s[j] - m);
-  for (int64_t d = 0; d < p.D; ++d) {
-    double acc = 0.0;
-    for (int64_t j = 0; j < nvis; ++j) acc += std::exp(s[j] - m) * V[j * p.D + d];
-    o_out[d] = acc / l;
+  for (int64_t j = 0; j < nvis; ++j) {
+    e[j] = std::exp(s[j] - m);
+    l += e[j];
   }
+  // O_d = sum_j e_j V_jd / l, each sum taken over j in ascending order
+  std::vector<double> acc(static_cast<size_t>(p.D), 0.0);
+  for (int64_t j = 0; j < nvis; ++j) {
+    const double ej = e[j];
+    const double* vj = &V[j * p.D];
+    for (int64_t d = 0; d < p.D; ++d) acc[d] += ej * vj[d];
+  }
+  for (int64_t d = 0; d < p.D; ++d) o_out[d] = acc[d] / l;
   return m + std::log(l);
 }
 
@@ -196,7 +204,9 @@ int oracle_attention_full(const uint16_t* q, const uint16_t* k, const uint16_t* 
 
 // The same definition for a list of (b, h, i) triples, one score row at a
 // time. rows: [nrows][3]; o_rows: [nrows][D]; lse_rows: [nrows]. Rows are
-// independent, so this is bit-identical to oracle_attention_full on them.
+// independent, so this is bit-identical to oracle_attention_full on them. The
+// rows of one (b, h) share that head's K and V widened to double once
+// (decoding is exact, so this changes no value).
 int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B, int64_t N,
                           int64_t H, int64_t D, double scale, int causal, int dtype, const int64_t* rows,
                           int64_t nrows, double* o_rows, double* lse_rows, int nthreads) {
@@ -206,24 +216,54 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
     const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
     if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= N) return 2;
   }
-  parallel_for(nrows, nthreads, [&](int64_t lo, int64_t hi) {
-    std::vector<double> qrow(static_cast<size_t>(D)), krow(static_cast<size_t>(D));
-    std::vector<double> s, Vvis;
-    for (int64_t r = lo; r < hi; ++r) {
-      const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
-      const int64_t nvis = visible_count(p, i);
-      s.assign(static_cast<size_t>(nvis), 0.0);
-      Vvis.assign(static_cast<size_t>(nvis * D), 0.0);
-      for (int64_t d = 0; d < D; ++d) qrow[d] = decode(q[at(p, b, i, h, d)], dtype);
-      for (int64_t j = 0; j < nvis; ++j) {
-        double dot = 0.0;
-        for (int64_t d = 0; d < D; ++d) dot += qrow[d] * decode(k[at(p, b, j, h, d)], dtype);
-        s[j] = scale * dot;
-        for (int64_t d = 0; d < D; ++d) Vvis[j * D + d] = decode(v[at(p, b, j, h, d)], dtype);
-      }
-      lse_rows[r] = finish_row(p, s.data(), nvis, Vvis, &o_rows[r * D]);
-    }
+  // the requested rows grouped by head (b, h), in request order within a head
+  std::vector<int64_t> order(static_cast<size_t>(nrows));
+  for (int64_t r = 0; r < nrows; ++r) order[r] = r;
+  std::stable_sort(order.begin(), order.end(), [&](int64_t x, int64_t y) {
+    return rows[3 * x] * H + rows[3 * x + 1] < rows[3 * y] * H + rows[3 * y + 1];
   });
+  std::vector<double> K, V;
+  for (int64_t g0 = 0; g0 < nrows;) {
+    const int64_t b = rows[3 * order[g0]], h = rows[3 * order[g0] + 1];
+    int64_t g1 = g0;
+    while (g1 < nrows && rows[3 * order[g1]] == b && rows[3 * order[g1] + 1] == h) ++g1;
+    widen_head(p, k, b, h, K);
+    widen_head(p, v, b, h, V);
+    parallel_for(g1 - g0, nthreads, [&](int64_t lo, int64_t hi) {
+      std::vector<double> qrow(static_cast<size_t>(D));
+      std::vector<double> s;
+      for (int64_t t = g0 + lo; t < g0 + hi; ++t) {
+        const int64_t r = order[t], i = rows[3 * r + 2];
+        const int64_t nvis = visible_count(p, i);
+        s.assign(static_cast<size_t>(nvis), 0.0);
+        for (int64_t d = 0; d < D; ++d) qrow[d] = decode(q[at(p, b, i, h, d)], dtype);
+        // s_j = scale * sum_d q_d k_jd, each sum over d in ascending order;
+        // four keys at a time only to give the CPU independent chains
+        int64_t j = 0;
+        for (; j + 4 <= nvis; j += 4) {
+          const double* k0 = &K[j * D];
+          double dot0 = 0.0, dot1 = 0.0, dot2 = 0.0, dot3 = 0.0;
+          for (int64_t d = 0; d < D; ++d) {
+            dot0 += qrow[d] * k0[d];
+            dot1 += qrow[d] * k0[D + d];
+            dot2 += qrow[d] * k0[2 * D + d];
+            dot3 += qrow[d] * k0[3 * D + d];
+          }
+          s[j] = scale * dot0;
+          s[j + 1] = scale * dot1;
+          s[j + 2] = scale * dot2;
+          s[j + 3] = scale * dot3;
+        }
+        for (; j < nvis; ++j) {
+          double dot = 0.0;
+          for (int64_t d = 0; d < D; ++d) dot += qrow[d] * K[j * D + d];
+          s[j] = scale * dot;
+        }
+        lse_rows[r] = finish_row(p, s.data(), nvis, V, &o_rows[r * D]);
+      }
+    });
+    g0 = g1;
+  }
   return 0;
 }
 
