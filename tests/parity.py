@@ -36,13 +36,14 @@ def passes(m: dict) -> bool:
 
 
 def sample_rows(B: int, H: int, N: int, per_head_random: int, seed: int = 0, heads: list | None = None,
-                block: int = 128) -> np.ndarray:
-    """(b, h, i) triples covering, for each chosen head, the first and last rows,
-    the rows on both sides of every `block` boundary, and random rows."""
+                block: int = 128, ends: int = 2) -> np.ndarray:
+    """(b, h, i) triples covering, for each chosen head (default: every head),
+    the first and last `ends` rows, the rows on both sides of every `block`
+    boundary, and `per_head_random` random rows."""
     rng = np.random.default_rng(seed)
     if heads is None:
         heads = [(b, h) for b in range(B) for h in range(H)]
-    edge = {0, 1, N - 2, N - 1}
+    edge = set(range(min(ends, N))) | set(range(max(0, N - ends), N))
     for t in range(block, N, block):
         edge.update((t - 1, t))
     edge = sorted(i for i in edge if 0 <= i < N)

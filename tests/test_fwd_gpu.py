@@ -74,14 +74,15 @@ def test_small_config_matches_golden_rows():
     assert passes(m), m
 
 
-def _check_sampled(w: Workload, per_head_random: int, max_heads: int | None = None):
+def _check_sampled(w: Workload, per_head_random: int = 64, ends: int = 256):
+    """Every (b, h) of a published configuration at full size: its first and
+    last `ends` rows, the rows on both sides of every 128-row tile boundary,
+    and `per_head_random` random rows, each computed one by one by the oracle
+    (exact per row); the whole output is checked to be written and finite."""
     q, k, v = make_qkv(w)
     o, lse = _run(q, k, v, w.softmax_scale, w.causal)
-    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    if max_heads is not None and len(heads) > max_heads:
-        idx = np.linspace(0, len(heads) - 1, max_heads).round().astype(int)
-        heads = [heads[i] for i in sorted(set(idx.tolist()))]
-    rows = sample_rows(w.B, w.H, w.N, per_head_random, seed=1, heads=heads)
+    rows = sample_rows(w.B, w.H, w.N, per_head_random, seed=1, ends=ends)
+    assert len({(b, h) for b, h, _ in rows.tolist()}) == w.B * w.H
     o_ref, lse_ref = oracle.attention_rows(bits(q), bits(k), bits(v), w.softmax_scale, w.causal, w.dtype, rows)
     m = metrics(o[rows[:, 0], rows[:, 2], rows[:, 1]], lse[rows[:, 0], rows[:, 1], rows[:, 2]], o_ref, lse_ref)
     assert passes(m), (w.name, m)
@@ -90,23 +91,23 @@ def _check_sampled(w: Workload, per_head_random: int, max_heads: int | None = No
     return m
 
 
-@pytest.mark.parametrize("name,per_head,max_heads", [
-    ("llama7b_b4h32n2048d128_causal", 8, None),
-    ("long_b1h32n8192d128_noncausal", 4, 8),
-    ("long_b1h32n8192d128_causal", 4, 8),
-    ("stress_b2h16n4093d64_fp16_causal", 8, None),
-    ("stress_hot_b2h16n4093d64_fp16_causal", 8, None),
-    ("sweep_n1024_noncausal", 4, 16),
-    ("sweep_n1024_causal", 4, 16),
-    ("sweep_n4096_noncausal", 4, 8),
-    ("sweep_n4096_causal", 4, 8),
-    ("sweep_n16384_noncausal", 2, 4),
-    ("sweep_n16384_causal", 2, 4),
-    ("sweep_n32768_noncausal", 1, 2),
-    ("sweep_n32768_causal", 1, 2),
+@pytest.mark.parametrize("name", [
+    "llama7b_b4h32n2048d128_causal",
+    "long_b1h32n8192d128_noncausal",
+    "long_b1h32n8192d128_causal",
+    "stress_b2h16n4093d64_fp16_causal",
+    "stress_hot_b2h16n4093d64_fp16_causal",
+    "sweep_n1024_noncausal",
+    "sweep_n1024_causal",
+    "sweep_n4096_noncausal",
+    "sweep_n4096_causal",
+    "sweep_n16384_noncausal",
+    "sweep_n16384_causal",
+    "sweep_n32768_noncausal",
+    "sweep_n32768_causal",
 ])
-def test_published_configs_sampled_rows(name, per_head, max_heads):
-    _check_sampled(WORKLOADS[name], per_head, max_heads)
+def test_published_configs_sampled_rows(name):
+    _check_sampled(WORKLOADS[name])
 
 
 def test_stress_logits_really_large():
@@ -212,3 +213,36 @@ def test_host_errors_do_not_launch():
     assert st == fa.FA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert bool((o == 3.0).all()) and bool((lse == 5.0).all())
+
+
+def test_memory_is_linear_in_n():
+    """The pages' memory claim (O(N), not O(N^2)): a forward at N = 32768
+    (B=1, H=16, D=128) runs while less device memory is free than ONE head's
+    N x N fp32 score matrix would take (4 GiB), and the call allocates nothing
+    (free device memory is the same before and after it)."""
+    w = WORKLOADS["sweep_n32768_noncausal"]
+    q, k, v = (t.to(DEV) for t in make_qkv(w))
+    o1, o2 = torch.empty_like(q), torch.full_like(q, float("nan"))
+    l1 = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=DEV)
+    l2 = torch.full_like(l1, float("nan"))
+    fa.fwd_into(q, k, v, o1, l1)  # warm-up, and the reference bits
+    assert fa.status_sync() == fa.FA_OK
+    torch.cuda.synchronize()
+    scores_one_head = w.N * w.N * 4
+    headroom = 2 << 30
+    free, _ = torch.cuda.mem_get_info()
+    filler = torch.empty(max(free - headroom, 0), dtype=torch.uint8, device=DEV)
+    try:
+        torch.cuda.synchronize()
+        free_before, _ = torch.cuda.mem_get_info()
+        assert free_before < scores_one_head, free_before
+        fa.fwd_into(q, k, v, o2, l2)
+        assert fa.status_sync() == fa.FA_OK
+        torch.cuda.synchronize()
+        free_after, _ = torch.cuda.mem_get_info()
+        assert free_after == free_before
+    finally:
+        del filler
+        torch.cuda.empty_cache()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))

@@ -4,30 +4,38 @@ Some callers must not allocate device memory on the call path (their GPU
 memory is reserved up front by another allocator, or they cannot handle an
 out-of-memory failure mid-request); this entry point keeps its partial
 results in a scratch buffer compiled into the library instead of a caller
-workspace. The test calls it through the C ABI twice in a row and compares
-each result with the workspace entry point fa_fwd_splitkv on the same inputs,
-within the parity tolerance used throughout the tests. It sits in its own
-file, collected last, and depends on no other test.
+workspace. The tests call it through the C ABI twice in a row (the scratch
+keeps the previous call's contents) and compare each result element by
+element with the fp64 oracle, at the tolerances used throughout the tests,
+and with the workspace entry point fa_fwd_splitkv. They cover the paired
+split-KV path (grouped heads packed into one tile), the unpaired one (one
+query head per K/V head), and a size whose automatic range count has to fall
+back to a smaller one so that the partial results fit the scratch; and they
+check that free device memory is the same before and after a call. The file
+sits last in collection order and depends on no other test.
 """
 
 import ctypes
 import math
 
+import numpy as np
 import pytest
 import torch
 
 import exact_attention_151_b200 as fa
+import oracle
+from exact_attention_151_b200.inputs import bits
 from tests.parity import metrics, passes
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _inputs(seed, B=1, Nq=4, Nk=6000, Hq=16, Hkv=4, D=128):
+def _inputs(seed, B, Nq, Nk, Hq, Hkv, D):
     g = torch.Generator().manual_seed(seed)
-    q = torch.randn(B, Nq, Hq, D, generator=g).to(torch.bfloat16).to(DEV)
-    k = torch.randn(B, Nk, Hkv, D, generator=g).to(torch.bfloat16).to(DEV)
-    v = torch.randn(B, Nk, Hkv, D, generator=g).to(torch.bfloat16).to(DEV)
+    q = torch.randn(B, Nq, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Nk, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Nk, Hkv, D, generator=g).to(torch.bfloat16)
     return q, k, v
 
 
@@ -40,20 +48,79 @@ def _noalloc_abi(q, k, v, o, lse, causal, num_splits=0):
         ctypes.c_float(1.0 / math.sqrt(D)), int(causal), fa.FA_BF16, num_splits, stream)
 
 
+def _oracle(q, k, v, causal):
+    """The oracle's packed form (bottom-right causal), as [B, Nq, Hq, D] and [B, Hq, Nq]."""
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, _ = k.shape
+    o, lse = oracle.attention_varlen(bits(q.reshape(B * Nq, Hq, D)), bits(k.reshape(B * Nk, Hkv, D)),
+                                     bits(v.reshape(B * Nk, Hkv, D)), np.arange(B + 1) * Nq, np.arange(B + 1) * Nk,
+                                     1 / math.sqrt(D), causal, "bf16")
+    return o.reshape(B, Nq, Hq, D), lse.reshape(Hq, B, Nq).transpose(1, 0, 2)
+
+
+SHAPES = [
+    # (B, Nq, Nk, Hq, Hkv, D): paired split-KV (4 query heads per K/V head packed into one tile)
+    (1, 4, 6000, 16, 4, 128),
+    # unpaired: one query head per K/V head, a single query, ragged last key tile
+    (1, 1, 6001, 8, 8, 128),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=["paired", "unpaired"])
 @pytest.mark.parametrize("causal", [True, False])
-def test_noalloc_matches_workspace_entry_point_twice(causal):
+def test_noalloc_matches_oracle_twice(shape, causal):
+    B, Nq, Nk, Hq, Hkv, D = shape
+    n, need = fa.splitkv_plan(B, Nq, Nk, Hq, D, Hkv=Hkv)
+    assert n > 1 and 0 < need <= fa.NOALLOC_SCRATCH_BYTES
     for call, seed in enumerate((101, 202)):  # two calls in a row: the scratch keeps the previous contents
-        q, k, v = _inputs(seed)
-        n, need = fa.splitkv_plan(q.shape[0], q.shape[1], k.shape[1], q.shape[2], q.shape[3], Hkv=k.shape[2])
-        assert n > 1 and 0 < need <= fa.NOALLOC_SCRATCH_BYTES
-        o_ref, lse_ref = fa.fwd_splitkv(q, k, v, causal=causal)
-        o = torch.full_like(q, float("nan"))
-        lse = torch.full_like(lse_ref, float("nan"))
-        assert _noalloc_abi(q, k, v, o, lse, causal) == fa.FA_OK
+        q, k, v = _inputs(seed + Nq, B, Nq, Nk, Hq, Hkv, D)
+        qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+        o = torch.full_like(qd, float("nan"))
+        lse = torch.full((B, Hq, Nq), float("nan"), device=DEV)
+        assert _noalloc_abi(qd, kd, vd, o, lse, causal) == fa.FA_OK
         assert fa.status_sync() == fa.FA_OK
-        m = metrics(o.cpu().double().numpy(), lse.cpu().double().numpy(), o_ref.cpu().double().numpy(),
-                    lse_ref.cpu().double().numpy())
+        o_ref, lse_ref = _oracle(q, k, v, causal)
+        m = metrics(o.cpu().double().numpy(), lse.cpu().double().numpy(), o_ref, lse_ref)
         assert passes(m), (call, m)
+        # and the workspace entry point on the same inputs agrees
+        o_ws, lse_ws = fa.fwd_splitkv(qd, kd, vd, causal=causal)
+        m2 = metrics(o.cpu().double().numpy(), lse.cpu().double().numpy(), o_ws.cpu().double().numpy(),
+                     lse_ws.cpu().double().numpy())
+        assert passes(m2), (call, m2)
+
+
+def test_noalloc_falls_back_to_a_range_count_that_fits():
+    """With num_splits = 0 the plan's range count needs more partial-result
+    memory than the scratch holds; the call uses the largest count that fits."""
+    B, Nq, Nk, Hq, Hkv, D = 1, 16, 65536, 32, 4, 128
+    n, need = fa.splitkv_plan(B, Nq, Nk, Hq, D, Hkv=Hkv)
+    assert need > fa.NOALLOC_SCRATCH_BYTES  # the automatic count does not fit
+    q, k, v = _inputs(7, B, Nq, Nk, Hq, Hkv, D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, Hq, Nq), float("nan"), device=DEV)
+    assert _noalloc_abi(qd, kd, vd, o, lse, True) == fa.FA_OK
+    assert fa.status_sync() == fa.FA_OK
+    o_ref, lse_ref = _oracle(q, k, v, True)
+    m = metrics(o.cpu().double().numpy(), lse.cpu().double().numpy(), o_ref, lse_ref)
+    assert passes(m), m
+
+
+def test_noalloc_call_leaves_free_memory_unchanged():
+    B, Nq, Nk, Hq, Hkv, D = SHAPES[0]
+    q, k, v = (t.to(DEV) for t in _inputs(5, B, Nq, Nk, Hq, Hkv, D))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), device=DEV)
+    assert _noalloc_abi(q, k, v, o, lse, True) == fa.FA_OK  # warm-up: the scratch address is looked up
+    assert fa.status_sync() == fa.FA_OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _noalloc_abi(q, k, v, o, lse, False) == fa.FA_OK
+    assert fa.status_sync() == fa.FA_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
