@@ -66,6 +66,10 @@ def _load():
         lib.oracle_attention_backward.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_double,
                                                   ctypes.c_int, ctypes.c_int, f64p, f64p, f64p, ctypes.c_int]
         lib.oracle_attention_backward.restype = ctypes.c_int
+        lib.oracle_attention_backward_varlen.argtypes = [u16p, u16p, u16p, u16p, i64p, i64p, i64, i64, i64, i64,
+                                                         ctypes.c_double, ctypes.c_int, ctypes.c_int, f64p, f64p,
+                                                         f64p, ctypes.c_int]
+        lib.oracle_attention_backward_varlen.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -184,6 +188,36 @@ def attention_backward(q, k, v, dout, scale: float, causal: bool, dtype: str, nt
         _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), int(nthreads or default_threads()))
     if rc:
         raise ValueError(f"oracle_attention_backward failed ({rc})")
+    return dq, dk, dv
+
+
+def attention_backward_varlen(q, k, v, dout, cu_q, cu_k, scale: float, causal: bool, dtype: str,
+                              nthreads: int | None = None):
+    """Gradients (dQ [total_q, Hq, D], dK and dV [total_k, Hkv, D], float64) of
+    sum(O * dO) through attention_varlen's definition: packed sequences,
+    grouped-query heads (a K/V head's gradient sums over the query heads that
+    read it), causal mask aligned at the bottom-right corner. Inputs are 16-bit
+    patterns: q and dout [total_q, Hq, D], k and v [total_k, Hkv, D]."""
+    q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
+    if q.ndim != 3 or k.ndim != 3 or k.shape != v.shape or q.shape[2] != k.shape[2] or dout.shape != q.shape:
+        raise ValueError("q and dout must be [total_q, Hq, D], k and v [total_k, Hkv, D]")
+    cu_q = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int64))
+    cu_k = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int64))
+    B = len(cu_q) - 1
+    if len(cu_k) != B + 1 or cu_q[-1] != q.shape[0] or cu_k[-1] != k.shape[0]:
+        raise ValueError("cu_seqlens do not match the tensors")
+    total_q, Hq, D = q.shape
+    Hkv = k.shape[1]
+    dq = np.empty((total_q, Hq, D), dtype=np.float64)
+    dk = np.empty(k.shape, dtype=np.float64)
+    dv = np.empty(k.shape, dtype=np.float64)
+    rc = _load().oracle_attention_backward_varlen(
+        _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16), _ptr(dout, ctypes.c_uint16),
+        _ptr(cu_q, ctypes.c_int64), _ptr(cu_k, ctypes.c_int64), B, Hq, Hkv, D, float(scale), int(bool(causal)),
+        DTYPE_CODES[dtype], _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),
+        int(nthreads or default_threads()))
+    if rc:
+        raise ValueError(f"oracle_attention_backward_varlen failed ({rc})")
     return dq, dk, dv
 
 

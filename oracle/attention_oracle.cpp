@@ -401,6 +401,107 @@ int oracle_attention_backward(const uint16_t* q, const uint16_t* k, const uint16
   return 0;
 }
 
+// Backward of oracle_attention_varlen (packed sequences, grouped-query heads,
+// causal mask aligned at the bottom-right corner), the same gradients as
+// oracle_attention_backward, per sequence b and query head h:
+//   P_ij, dP_ij, D_i, dS_ij  as there, over the keys visible to query i
+//                            (P_ij = dS_ij = 0 elsewhere; a query with no
+//                            visible key has P = 0 and dQ = 0)
+//   dQ_i  (head h)           = scale * sum_j dS_ij K_j
+//   dK_j  (K/V head hk)      = scale * sum_{h in group(hk)} sum_i dS^h_ij Q^h_i
+//   dV_j  (K/V head hk)      = sum_{h in group(hk)} sum_i P^h_ij dO^h_i
+// where group(hk) are the query heads hk G .. hk G + G - 1 (G = Hq / Hkv)
+// that read K/V head hk: each K/V element serves every head of its group, so
+// its gradient is the sum over them (taken in ascending h, each head's sum
+// over i first). Layouts as oracle_attention_varlen: q, dout, dq
+// [total_q, Hq, D]; k, v, dk, dv [total_k, Hkv, D]; gradients in double.
+int oracle_attention_backward_varlen(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                                     const int64_t* cu_q, const int64_t* cu_k, int64_t B, int64_t Hq, int64_t Hkv,
+                                     int64_t D, double scale, int causal, int dtype, double* dq, double* dk,
+                                     double* dv, int nthreads) {
+  if (!q || !k || !v || !dout || !cu_q || !cu_k || !dq || !dk || !dv || B < 0 || Hq < 1 || Hkv < 1 || D < 1 ||
+      Hq % Hkv != 0 || (dtype != 0 && dtype != 1))
+    return 1;
+  for (int64_t b = 0; b < B; ++b)
+    if (cu_q[b + 1] < cu_q[b] || cu_k[b + 1] < cu_k[b] || cu_q[0] != 0 || cu_k[0] != 0) return 2;
+  const int64_t group = Hq / Hkv;
+  // widen rows r0 .. r0+n-1 of head h of a [total, heads, D] tensor to [n][D]
+  auto widen = [&](const uint16_t* src, int64_t heads, int64_t h, int64_t r0, int64_t n, std::vector<double>& dst) {
+    dst.resize(static_cast<size_t>(n * D));
+    for (int64_t r = 0; r < n; ++r)
+      for (int64_t d = 0; d < D; ++d) dst[r * D + d] = decode(src[((r0 + r) * heads + h) * D + d], dtype);
+  };
+  std::vector<double> Q, K, V, dO, P, dS, dKacc, dVacc;
+  for (int64_t b = 0; b < B; ++b) {
+    const int64_t q0 = cu_q[b], nq = cu_q[b + 1] - q0, k0 = cu_k[b], nk = cu_k[b + 1] - k0;
+    for (int64_t hk = 0; hk < Hkv; ++hk) {
+      widen(k, Hkv, hk, k0, nk, K);
+      widen(v, Hkv, hk, k0, nk, V);
+      dKacc.assign(static_cast<size_t>(nk * D), 0.0);
+      dVacc.assign(static_cast<size_t>(nk * D), 0.0);
+      for (int64_t h = hk * group; h < (hk + 1) * group; ++h) {
+        widen(q, Hq, h, q0, nq, Q);
+        widen(dout, Hq, h, q0, nq, dO);
+        P.assign(static_cast<size_t>(nq * nk), 0.0);
+        dS.assign(static_cast<size_t>(nq * nk), 0.0);
+        // rows: P, O, D, dP, dS, then dQ
+        parallel_for(nq, nthreads, [&](int64_t lo, int64_t hi) {
+          std::vector<double> s(static_cast<size_t>(nk)), orow(static_cast<size_t>(D));
+          for (int64_t i = lo; i < hi; ++i) {
+            int64_t nvis = nk;
+            if (causal) nvis = std::min(nk, std::max<int64_t>(0, i + nk - nq + 1));
+            double* dqrow = &dq[((q0 + i) * Hq + h) * D];
+            if (nvis == 0) {
+              for (int64_t d = 0; d < D; ++d) dqrow[d] = 0.0;
+              continue;
+            }
+            for (int64_t j = 0; j < nvis; ++j) {
+              double dot = 0.0;
+              for (int64_t d = 0; d < D; ++d) dot += Q[i * D + d] * K[j * D + d];
+              s[j] = scale * dot;
+            }
+            Problem p{q, k, v, 1, nk, 1, D, scale, causal, dtype};
+            const double lse = finish_row(p, s.data(), nvis, V, orow.data());
+            double Di = 0.0;
+            for (int64_t d = 0; d < D; ++d) Di += dO[i * D + d] * orow[d];
+            for (int64_t j = 0; j < nvis; ++j) {
+              const double pij = std::exp(s[j] - lse);
+              double dpij = 0.0;
+              for (int64_t d = 0; d < D; ++d) dpij += dO[i * D + d] * V[j * D + d];
+              P[i * nk + j] = pij;
+              dS[i * nk + j] = pij * (dpij - Di);
+            }
+            for (int64_t d = 0; d < D; ++d) {
+              double acc = 0.0;
+              for (int64_t j = 0; j < nk; ++j) acc += dS[i * nk + j] * K[j * D + d];
+              dqrow[d] = scale * acc;
+            }
+          }
+        });
+        // this head's share of dK, dV
+        parallel_for(nk, nthreads, [&](int64_t lo, int64_t hi) {
+          for (int64_t j = lo; j < hi; ++j)
+            for (int64_t d = 0; d < D; ++d) {
+              double ak = 0.0, av = 0.0;
+              for (int64_t i = 0; i < nq; ++i) {
+                ak += dS[i * nk + j] * Q[i * D + d];
+                av += P[i * nk + j] * dO[i * D + d];
+              }
+              dKacc[j * D + d] += ak;
+              dVacc[j * D + d] += av;
+            }
+        });
+      }
+      for (int64_t j = 0; j < nk; ++j)
+        for (int64_t d = 0; d < D; ++d) {
+          dk[((k0 + j) * Hkv + hk) * D + d] = scale * dKacc[j * D + d];
+          dv[((k0 + j) * Hkv + hk) * D + d] = dVacc[j * D + d];
+        }
+    }
+  }
+  return 0;
+}
+
 // The handbook's tiled online-softmax routine, in fp64, one (b, h) at a time.
 // For every query block [qs, qe) and every key block [ks, ke) (both cut at
 // block_size, the last one truncated at N):
