@@ -16,7 +16,8 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "bwd", "bwd_workspace_size", "status_sync", "FaError", "library_path", "load_library",
+__all__ = ["fwd", "fwd_into", "fwd_varlen", "fwd_splitkv", "splitkv_plan", "fwd_ptr", "bwd", "bwd_varlen",
+           "bwd_workspace_size", "status_sync", "FaError", "library_path", "load_library",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_MISALIGNED", "FA_ERR_CUDA",
            "FA_ERR_TIMEOUT", "FA_ERR_DEVICE_CHECK", "EXPORTED_SYMBOLS", "load_checking_library"]
 
@@ -34,7 +35,7 @@ FA_FP16 = 1
 # Every entry point declared in include/fa.h.
 EXPORTED_SYMBOLS = ("fa_status_string", "fa_last_error", "fa_fwd", "fa_fwd_gqa", "fa_fwd_varlen",
                     "fa_fwd_splitkv", "fa_fwd_splitkv_plan", "fa_fwd_splitkv_noalloc", "fa_status_sync",
-                    "fa_fwd_debug", "fa_bwd", "fa_bwd_workspace_size")
+                    "fa_fwd_debug", "fa_bwd", "fa_bwd_gqa", "fa_bwd_varlen", "fa_bwd_workspace_size")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_HERE, "libfa_b200.so")
@@ -107,6 +108,12 @@ def _open(path):
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, i32, i32, vp,
                            ctypes.c_size_t, vp]
     lib.fa_bwd.restype = i32
+    lib.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i32,
+                               i32, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd_gqa.restype = i32
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64,
+                                  ctypes.c_float, i32, i32, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd_varlen.restype = i32
     lib.fa_status_sync.argtypes = [vp]
     lib.fa_status_sync.restype = i32
     return lib
@@ -328,19 +335,24 @@ def bwd_workspace_size(B: int, N: int, H: int) -> int:
 
 def bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False, dq=None, dk=None, dv=None,
         workspace=None):
-    """Gradients (dq, dk, dv) of sum(O * dout) for the forward's q, k, v [B,N,H,D], o and lse.
+    """Gradients (dq, dk, dv) of sum(O * dout) for the forward's q [B,Nq,Hq,D], k, v [B,Nk,Hkv,D], o and lse.
 
     ``o`` and ``lse`` are what fwd returned for the same q, k, v, scale and
-    causal. dq/dk/dv (like q) and ``workspace`` (CUDA uint8, at least
-    bwd_workspace_size(B, N, H) bytes) are allocated here if omitted.
+    causal (with Nk != Nq the causal mask is aligned at the bottom-right
+    corner; with Hkv < Hq a K/V head's gradient sums over the query heads that
+    read it). dq (like q), dk, dv (like k) and ``workspace`` (CUDA uint8, at
+    least bwd_workspace_size(B, Nq, Hq) bytes) are allocated here if omitted.
     """
     import torch
 
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape or dout.shape != q.shape:
-        raise ValueError("q, k, v, o and dout must all be [B, N, H, D]")
-    B, N, H, D = q.shape
-    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
-        raise ValueError("lse must be float32 [B, H, N]")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("q, o, dout must be [B, Nq, Hq, D] and k, v [B, Nk, Hkv, D]")
+    B, Nq, Hq, D = q.shape
+    Bk, Nk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q and k/v disagree on batch or head dimension")
+    if tuple(lse.shape) != (B, Hq, Nq) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, Hq, Nq]")
     for t in (k, v, o, dout):
         if t.dtype != q.dtype:
             raise TypeError("q, k, v, o and dout must share one dtype")
@@ -348,21 +360,71 @@ def bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False,
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    for t in (dq, dk, dv):
-        if t.shape != q.shape or t.dtype != q.dtype:
-            raise ValueError("dq, dk and dv must be like q")
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    if dq.shape != q.shape or dq.dtype != q.dtype or dk.shape != k.shape or dv.shape != k.shape or \
+            dk.dtype != q.dtype or dv.dtype != q.dtype:
+        raise ValueError("dq must be like q, dk and dv like k")
     with torch.cuda.device(q.device):
-        need = bwd_workspace_size(B, N, H)
+        need = bwd_workspace_size(B, Nq, Hq)
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
         _check_cuda(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace)
         stream = torch.cuda.current_stream(q.device).cuda_stream
-        st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D,
-                                   ctypes.c_float(float(scale)), int(bool(causal)), code, workspace.data_ptr(),
-                                   workspace.numel() * workspace.element_size(), stream)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+        tail = (ctypes.c_float(float(scale)), int(bool(causal)), code, workspace.data_ptr(),
+                workspace.numel() * workspace.element_size(), stream)
+        if Nq == Nk and Hq == Hkv:
+            st = load_library().fa_bwd(*args, B, Nq, Hq, D, *tail)
+        else:
+            st = load_library().fa_bwd_gqa(*args, B, Nq, Nk, Hq, Hkv, D, *tail)
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+               scale: float | None = None, causal: bool = False, dq=None, dk=None, dv=None, workspace=None):
+    """Backward of fwd_varlen: q, o, dout [total_q, Hq, D]; k, v [total_k, Hkv, D];
+    lse fp32 [Hq, total_q] as fwd_varlen returned it; cu_seqlens_* int32 CUDA
+    tensors of B+1 offsets. Returns (dq like q, dk and dv like k). Inconsistent
+    offsets are reported by status_sync() as FA_ERR_INVALID_ARG."""
+    import torch
+
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape or \
+            q.shape[2] != k.shape[2]:
+        raise ValueError("q, o, dout must be [total_q, Hq, D] and k, v [total_k, Hkv, D]")
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    if tuple(lse.shape) != (Hq, total_q) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [Hq, total_q]")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_k.shape != cu_seqlens_q.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must be 1-D with B+1 entries")
+    for t in (k, v, o, dout):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, o and dout must share one dtype")
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    with torch.cuda.device(q.device):
+        need = bwd_workspace_size(B, max_seqlen_q, Hq)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        _check_cuda(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace,
+                    cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k)
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        st = load_library().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                          cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                                          int(max_seqlen_k), total_q, total_k, Hq, Hkv, D,
+                                          ctypes.c_float(float(scale)), int(bool(causal)), _dtype_code(q),
+                                          workspace.data_ptr(), workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd_varlen")
     return dq, dk, dv

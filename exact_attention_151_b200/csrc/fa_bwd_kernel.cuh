@@ -73,17 +73,60 @@ struct Cfg {
   static_assert(256 + 2 * D <= 512, "TMEM budget");
 };
 
+// Shapes: q, o, dO, dQ [B, Nq, Hq, D]; k, v, dK, dV [B, Nk, Hkv, D] (dense), or
+// packed sequences [total_q, Hq, D] and [total_k, Hkv, D] where sequence b
+// owns query rows cu_q[b] .. cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1.
+// Query head h reads K/V head h / G (G = Hq / Hkv). Causal: key j is visible
+// to query i iff j <= i + delta, delta = nk - nq (aligned at the bottom-right
+// corner) for the sequence's lengths nq, nk.
 struct Params {
-  const float* ws_d;    // [B*H, Npad]: -D_i = -dO_i . O_i (0 on pad rows)
-  const float* ws_l;    // [B*H, Npad]: -LSE_i * log2(e) (-inf on pad rows)
+  const int* cu_q;      // packed sequences: B+1 query row offsets (device memory); dense: null
+  const int* cu_k;      // packed sequences: B+1 key row offsets
+  int total_q, total_k; // rows of the query-side and key-side tensors
+  const float* ws_d;    // [B*Hq, Npad]: -D_i = -dO_i . O_i (0 on pad rows)
+  const float* ws_l;    // [B*Hq, Npad]: -LSE_i * log2(e) (-inf on pad rows and rows that see no key)
   uint16_t* out0;       // query side: dQ;   key side: dK
   uint16_t* out1;       // key side: dV
-  int N, H, BH, Npad, n_tiles;
+  int Nq, Nk;           // dense: the lengths; packed: upper bounds of every sequence's lengths
+  int Hq, Hkv, G;
+  int BH;               // heads of this kernel's grid: B * Hq (query side) or B * Hkv (key side)
+  int Npad;             // Nq rounded up to whole 128-row tiles
+  int n_tiles;          // tiles per head of this kernel's grid: query tiles (query side) or key tiles (key side)
   float scale_log2;     // scale * log2(e)
   float scale;
   int causal;
   unsigned long long wait_limit_ns;
 };
+
+// One sequence's rows and lengths as a CTA sees them.
+struct Seq {
+  int q0, nq, k0, nk;  // query rows q0 .. q0+nq-1, key rows k0 .. k0+nk-1
+  int n_qt, n_kt;      // their 128-row tiles
+  int delta;           // nk - nq: causal offset
+  bool ok;             // packed offsets consistent
+};
+
+__device__ __forceinline__ Seq resolve_seq(const Params& prm, int b) {
+  Seq sq;
+  if (prm.cu_q != nullptr) {
+    sq.q0 = prm.cu_q[b];
+    sq.nq = prm.cu_q[b + 1] - sq.q0;
+    sq.k0 = prm.cu_k[b];
+    sq.nk = prm.cu_k[b + 1] - sq.k0;
+    sq.ok = sq.q0 >= 0 && sq.nq >= 0 && sq.nq <= prm.Nq && static_cast<int64_t>(sq.q0) + sq.nq <= prm.total_q &&
+            sq.k0 >= 0 && sq.nk >= 0 && sq.nk <= prm.Nk && static_cast<int64_t>(sq.k0) + sq.nk <= prm.total_k;
+  } else {
+    sq.q0 = b * prm.Nq;
+    sq.nq = prm.Nq;
+    sq.k0 = b * prm.Nk;
+    sq.nk = prm.Nk;
+    sq.ok = true;
+  }
+  sq.n_qt = (sq.nq + kTile - 1) / kTile;
+  sq.n_kt = (sq.nk + kTile - 1) / kTile;
+  sq.delta = sq.nk - sq.nq;
+  return sq;
+}
 
 // -D_i and -LSE_i log2(e) per row into the tile-padded workspace (negated:
 // the kernels add them). Blocks below n_real_blocks read O and dO in memory
@@ -122,7 +165,9 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
       const int i = static_cast<int>(bi % N);
       const int64_t bh = (bi / N) * H + h;
       ws_d[bh * Npad + i] = -acc;
-      ws_l[bh * Npad + i] = -lse[bh * N + i] * 1.44269504088896340736f;
+      // a row that sees no key has LSE = -inf: its weights are 0, not exp(+inf)
+      const float l = lse[bh * N + i];
+      ws_l[bh * Npad + i] = l == -INFINITY ? -INFINITY : -l * 1.44269504088896340736f;
     }
   } else {
     const int pad = Npad - N;
@@ -135,10 +180,74 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
   }
 }
 
+// The same for packed sequences: O, dO [total_q, H, D], LSE [H, total_q],
+// the workspace [B*H, Npad] per (sequence, head). Row r belongs to the sequence
+// b with cu_q[b] <= r < cu_q[b+1] (binary search over the offsets); blocks from
+// n_real_blocks on fill each (sequence, head)'s pad rows nq .. Npad-1. With
+// inconsistent offsets nothing outside the workspace is written (the main
+// kernels report them).
+template <int D, bool FP16>
+__global__ void __launch_bounds__(256) fa_bwd_prep_varlen_kernel(const uint16_t* __restrict__ o,
+                                                                 const uint16_t* __restrict__ dout,
+                                                                 const float* __restrict__ lse,
+                                                                 float* __restrict__ ws_d, float* __restrict__ ws_l,
+                                                                 const int* __restrict__ cu_q, int B, int H,
+                                                                 int total_q, int Npad, unsigned n_real_blocks) {
+  constexpr int kLanes = D / 8;
+  constexpr int kRowsPerBlock = 256 / kLanes;
+  if (blockIdx.x < n_real_blocks) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanes;  // r H + h
+    const int sub = threadIdx.x % kLanes;
+    const bool valid = row < static_cast<int64_t>(total_q) * H;
+    float acc = 0.f;
+    if (valid) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
+      const uint4 y = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 a = unpack2<FP16>(xs[k]);
+        const float2 c = unpack2<FP16>(ys[k]);
+        acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+      }
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid && sub == 0) {
+      const int h = static_cast<int>(row % H);
+      const int r = static_cast<int>(row / H);
+      int lo = 0, hi = B;  // last b with cu_q[b] <= r
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (cu_q[mid] <= r) lo = mid; else hi = mid;
+      }
+      const int i = r - cu_q[lo];
+      if (i >= 0 && i < Npad) {
+        const int64_t at = (static_cast<int64_t>(lo) * H + h) * Npad + i;
+        ws_d[at] = -acc;
+        const float l = lse[static_cast<int64_t>(h) * total_q + r];
+        ws_l[at] = l == -INFINITY ? -INFINITY : -l * 1.44269504088896340736f;
+      }
+    }
+  } else {
+    const int64_t p = static_cast<int64_t>(blockIdx.x - n_real_blocks) * 256 + threadIdx.x;
+    if (p < static_cast<int64_t>(B) * H * Npad) {
+      const int b = static_cast<int>(p / (static_cast<int64_t>(H) * Npad));
+      const int i = static_cast<int>(p % Npad);
+      const int nq = cu_q[b + 1] - cu_q[b];
+      if (i >= nq || nq < 0) {
+        ws_d[p] = 0.f;
+        ws_l[p] = -INFINITY;
+      }
+    }
+  }
+}
+
 // Phase A for one thread's half row: p = 2^(s c + nl) for the 64 scores of
 // TMEM columns kColS + 64h .. (two 32-column chunks). nl is -LSE log2(e):
 // per row (query side, `nl_row`) or per column from shared memory (key side,
-// `nl_col`). MASKED tiles (the causal diagonal or the ragged tail) zero the
+// `nl_col`). MASKED tiles (causal tiles the diagonal cuts, key j visible to
+// query i iff j <= i + delta, or the ragged tail of the keys) zero the
 // invisible entries through the exponent and use the MUFU exp only; other
 // tiles send every second pair through the FMA-pipe polynomial (the
 // backward's exp work per tile is MUFU-bound at one exp unit per SM
@@ -146,7 +255,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
 // 16-bit weights are stored to the half's first 32 columns (key side: P^T).
 template <bool FP16, bool KV_SIDE, bool MASKED, bool PACK>
 __device__ __forceinline__ void phase_a(uint32_t t_s, float c, float nl_row, const float* nl_col, int first_col,
-                                        int row_abs, int n_valid, int causal, float (&p)[64]) {
+                                        int row_abs, int n_valid, int causal, int delta, float (&p)[64]) {
   const float2 c2 = make_float2(c, c);
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
@@ -170,12 +279,12 @@ __device__ __forceinline__ void phase_a(uint32_t t_s, float c, float nl_row, con
       if constexpr (MASKED) {
         const int c0 = first_col + e;  // column index (query on the key side, key on the query side)
         bool v0, v1;
-        if constexpr (KV_SIDE) {  // row = key row_abs; pad queries already carry -inf through nl
-          v0 = !causal || c0 >= row_abs;
-          v1 = !causal || c0 + 1 >= row_abs;
-        } else {                  // row = query row_abs
-          v0 = c0 < n_valid && (!causal || c0 <= row_abs);
-          v1 = c0 + 1 < n_valid && (!causal || c0 + 1 <= row_abs);
+        if constexpr (KV_SIDE) {  // row = key row_abs, column = query c0; pad queries carry -inf through nl
+          v0 = !causal || row_abs <= c0 + delta;
+          v1 = !causal || row_abs <= c0 + 1 + delta;
+        } else {                  // row = query row_abs, column = key c0 (n_valid keys)
+          v0 = c0 < n_valid && (!causal || c0 <= row_abs + delta);
+          v1 = c0 + 1 < n_valid && (!causal || c0 + 1 <= row_abs + delta);
         }
         x.x = v0 ? x.x : -INFINITY;
         x.y = v1 ? x.y : -INFINITY;
@@ -226,9 +335,12 @@ __device__ __forceinline__ void phase_b(uint32_t t_dp, uint32_t t_out, float nd_
   }
 }
 
-// Key side: a tile of 128 keys; X1 = K, X2 = V stay in shared memory, (Q_t,
-// dO_t) stream over query tiles t = first .. n_tiles-1 through a two-stage
-// ring, each stage with the tile's -LSE log2(e) and -D; out0 = dK, out1 = dV.
+// Key side: a tile of 128 keys of one K/V head; X1 = K, X2 = V stay in shared
+// memory, and (Q_t, dO_t) stream through a two-stage ring, each stage with the
+// tile's -LSE log2(e) and -D, as items u = (g, t): for each of the G query
+// heads g that read this K/V head, the query tiles t whose queries see some
+// key of the tile. dK and dV accumulate over all items in TMEM (a fixed order,
+// no atomics); out0 = dK, out1 = dV.
 // TMEM holds one S^T / dP^T pair beside the two accumulators, so the MMA warp
 // interleaves consecutive tiles, S(0) dP(0) | dV(t) S(t+1) dK(t) dP(t+1) | ...,
 // issuing each accumulating product per half as soon as that half is in TMEM.
@@ -250,12 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int N = prm.N;
   const int causal = prm.causal;
-  // CTA -> (bh, key tile). Causal work per tile is uneven (key tile j streams
-  // n_tiles - j query tiles): CTAs go in groups of kGroup heads, heaviest
-  // tiles first within a group, so the last wave holds the short ones and a
-  // group's Q/dO stay L2-resident. Non-causal: head-major.
+  // CTA -> (bh, key tile), bh = b * Hkv + hk. Causal work per tile is uneven
+  // (later key tiles are seen by fewer query tiles): CTAs go in groups of
+  // kGroup heads, heaviest tiles first within a group, so the last wave holds
+  // the short ones and a group's Q/dO stay L2-resident. Non-causal: head-major.
   int tile, bh;
   if (causal) {
     const int per_group = kGroup * prm.n_tiles;
@@ -269,10 +380,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
     bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
   }
-  const int b = bh / prm.H, h = bh % prm.H;
-  // streamed query tiles (causal ? tile : 0) .. n_tiles-1
-  const int t_first = causal ? tile : 0;
-  const int n_t = prm.n_tiles - t_first;
+  const int b = bh / prm.Hkv, hk = bh % prm.Hkv;
+  const Seq sq = resolve_seq(prm, b);
+  if (!sq.ok) {  // inconsistent packed offsets: report, touch nothing
+    if (threadIdx.x == 0) atomicOr(&g_status_word, 2u);
+    return;
+  }
+  if (tile >= sq.n_kt) return;  // key tile past the end of this sequence
+  // Query tiles that see some key of this tile: from the one holding the
+  // first query i with i + delta >= tile * 128 (causal) to the last.
+  int t_first = 0;
+  if (causal) {
+    const int i0 = tile * kTile - sq.delta;
+    t_first = i0 <= 0 ? 0 : i0 / kTile;
+  }
+  const int per_head = max(0, sq.n_qt - t_first);
+  const int n_t = prm.G * per_head;  // streamed items; item u: query head hk G + u / per_head, tile t_first + u % per_head
+  auto item_head = [&](int u) { return hk * prm.G + u / per_head; };
+  auto item_tile = [&](int u) { return t_first + u % per_head; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarX), 1);
@@ -300,9 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, prm.wait_limit_ns};
-  const int row0 = b * N;  // first row of this (b) in the [B*N, H, D] views
+  const int krow0 = sq.k0;  // first row of this sequence in the [rows, Hkv, D] views
+  const int qrow0 = sq.q0;  // and in the [rows, Hq, D] views
 
   if (warp == kLoad) {
+    if (n_t > 0) {
     // ------------------------------------------------------------ loader (converged warp)
     if (lane == 0) {
       tma_prefetch_desc(&tm_x1);
@@ -313,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
     for (int hf = 0; hf < C::kHalves; ++hf) {
-      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_x1, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
-      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_x2, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
+      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_x1, hf * 64, hk, krow0 + tile * kTile, bar(C::kBarX));
+      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_x2, hf * 64, hk, krow0 + tile * kTile, bar(C::kBarX));
     }
     int issued = 0;
     for (int t = 0; t < n_t; ++t) {
@@ -322,15 +449,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t >= C::kStages &&
           !warp_wait_bar(bar(C::kBarYEmpty + s), static_cast<uint32_t>(((t / C::kStages) & 1) ^ 1), wc))
         break;
-      const int row = row0 + (t_first + t) * kTile;
+      const int hq = item_head(t), tq = item_tile(t);
+      const int row = qrow0 + tq * kTile;
       mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + C::kWsBytes);
       for (int hf = 0; hf < C::kHalves; ++hf) {
-        tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, h, row, bar(C::kBarYFull + s));
-        tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, h, row, bar(C::kBarYFull + s));
+        tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, hq, row, bar(C::kBarYFull + s));
+        tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, hq, row, bar(C::kBarYFull + s));
       }
       {
         // this query tile's -LSE log2(e) and -D ride with Q_t and dO_t
-        const int64_t ws_row = static_cast<int64_t>(bh) * prm.Npad + (t_first + t) * kTile;
+        const int64_t ws_row = (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Npad + tq * kTile;
         bulk_load_elect(ws_stage(s), prm.ws_l + ws_row, kTile * 4, bar(C::kBarYFull + s));
         bulk_load_elect(ws_stage(s) + kTile * 4, prm.ws_d + ws_row, kTile * 4, bar(C::kBarYFull + s));
       }
@@ -342,7 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = s + ((issued - 1 - s) / C::kStages) * C::kStages;
       drain_wait(bar(C::kBarYFull + s), static_cast<uint32_t>((tl / C::kStages) & 1));
     }
+    }
   } else if (warp == kMma) {
+    if (n_t > 0) {
     // ------------------------------------------------------------ MMA issue (converged warp)
     constexpr uint32_t idesc_score = instr_desc_f16(kTile, kTile, FP16, false);
     constexpr uint32_t idesc_acc = instr_desc_f16(kTile, D, FP16, true);
@@ -423,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_elect(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0);
     }
+    }
   } else {
     // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
     const int wg = warp / 4;                  // column half of every score tile
@@ -437,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_ds = t_dp;  // dS^T pairs over the first half of this half of dP^T
     bool ok = true;
     for (int t = 0; t < n_t; ++t) {
-      const int cbase = (t_first + t) * kTile;  // first column (key, or query) of this tile
+      const int cbase = item_tile(t) * kTile;  // first query (column) of this item's tile
       const int first_col = cbase + 64 * wg;
       const uint32_t ph = static_cast<uint32_t>(t & 1);
       // key side: this tile's -LSE log2(e) and -D for the warpgroup's 64 query
@@ -445,7 +576,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = t % C::kStages;
       const float* nl_col = reinterpret_cast<const float*>(smem + C::kWsOff + s * C::kWsBytes) + 64 * wg;
       const float* nd_col = nl_col + kTile;
-      const bool masked = (causal && cbase == tile * kTile) || cbase + kTile > N;
+      // masked: the causal boundary cuts the tile (its last key is not seen by
+      // its first query), or the queries run out
+      const bool masked = (causal && tile * kTile + kTile - 1 > cbase + sq.delta) || cbase + kTile > sq.nq;
       ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
       if (!ok) break;
       ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
@@ -453,9 +586,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float p[64];
       if (masked) {
-        phase_a<FP16, true, true, true>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
+        phase_a<FP16, true, true, true>(t_s, c, nl_row, nl_col, first_col, r_abs, sq.nq, causal, sq.delta, p);
       } else {
-        phase_a<FP16, true, false, true>(t_s, c, nl_row, nl_col, first_col, r_abs, N, causal, p);
+        phase_a<FP16, true, false, true>(t_s, c, nl_row, nl_col, first_col, r_abs, sq.nq, causal, sq.delta, p);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -468,12 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::kBarB + wg));
     }
-    if (ok) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
+    if (ok && n_t > 0) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
     if (ok) {
       tc_fence_after();
-      // warpgroup 0 writes dK (scaled), warpgroup 1 dV
-      const bool row_valid = r_abs < N && index_ok(static_cast<int64_t>(b) * prm.H + h < prm.BH && h < prm.H);
-      uint16_t* dst_row = (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D;
+      // warpgroup 0 writes dK (scaled), warpgroup 1 dV; no query sees these
+      // keys when there were no items: both are 0
+      const bool row_valid =
+          r_abs < sq.nk && index_ok(static_cast<int64_t>(sq.k0) + r_abs < prm.total_k && hk < prm.Hkv);
+      uint16_t* dst_row = (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(sq.k0) + r_abs) * prm.Hkv + hk) * D;
       const float mul = wg == 1 ? 1.f : prm.scale;
       constexpr int kCols = D;
       const uint32_t acc = tmem + lane_base + (wg == 0 ? C::kColAcc0 : C::kColAcc1);
@@ -486,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul);
+          pk[k] = n_t > 0 ? pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul) : 0u;
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + col0 + q * 32);
 #pragma unroll
@@ -561,10 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int N = prm.N;
   const int causal = prm.causal;
-  // CTA -> (bh, query tile): causal in groups of kGroup heads, heaviest
-  // (latest) query tiles first; non-causal head-major.
+  // CTA -> (bh, query tile), bh = b * Hq + h: causal in groups of kGroup
+  // heads, heaviest (latest) query tiles first; non-causal head-major.
   int tile, bh;
   if (causal) {
     const int per_group = kGroup * prm.n_tiles;
@@ -577,8 +711,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
     bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
   }
-  const int b = bh / prm.H, h = bh % prm.H;
-  const int n_t = causal ? tile + 1 : prm.n_tiles;  // key tiles 0 .. n_t-1
+  const int b = bh / prm.Hq, h = bh % prm.Hq;
+  const int hk = h / prm.G;  // the K/V head this query head reads
+  const Seq sq = resolve_seq(prm, b);
+  if (!sq.ok) {  // inconsistent packed offsets: report, touch nothing
+    if (threadIdx.x == 0) atomicOr(&g_status_word, 2u);
+    return;
+  }
+  if (tile >= sq.n_qt) return;  // query tile past the end of this sequence
+  // key tiles 0 .. n_t-1: all of them, or (causal) up to the one holding the
+  // last key the tile's last query sees; none if no query of the tile sees a key
+  int n_t = sq.n_kt;
+  if (causal) {
+    const int last_key = tile * kTile + kTile - 1 + sq.delta;
+    n_t = last_key < 0 ? 0 : min(sq.n_kt, last_key / kTile + 1);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarX), 1);
@@ -609,9 +756,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, prm.wait_limit_ns};
-  const int row0 = b * N;
+  const int qrow0 = sq.q0;  // first row of this sequence in the [rows, Hq, D] views
+  const int krow0 = sq.k0;  // and in the [rows, Hkv, D] views
 
   if (warp == kLoad) {
+    if (n_t > 0) {
     // ------------------------------------------------------------ loader (converged warp)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -622,19 +771,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
     for (int hf = 0; hf < C::kHalves; ++hf) {
-      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
-      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_do, hf * 64, h, row0 + tile * kTile, bar(C::kBarX));
+      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, qrow0 + tile * kTile, bar(C::kBarX));
+      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_do, hf * 64, h, qrow0 + tile * kTile, bar(C::kBarX));
     }
     int nk = 0, nv = 0;  // K and V tiles issued
     for (int t = 0; t < n_t; ++t) {
-      const int row = row0 + t * kTile;
+      const int row = krow0 + t * kTile;
       const int sk = t % C::kKStages;
       if (t >= C::kKStages &&
           !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((t / C::kKStages) & 1) ^ 1), wc))
         break;
       mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
       for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, h, row, bar(C::kBarKFull + sk));
+        tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, row, bar(C::kBarKFull + sk));
       nk = t + 1;
       const int sv = t % C::kVStages;
       if (t >= C::kVStages &&
@@ -642,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
       for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, h, row, bar(C::kBarVFull + sv));
+        tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, row, bar(C::kBarVFull + sv));
       nv = t + 1;
     }
     // let the copies this warp issued land before shared memory is released
@@ -655,7 +804,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = s + ((nv - 1 - s) / C::kVStages) * C::kVStages;
       drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((tl / C::kVStages) & 1));
     }
+    }
   } else if (warp == kMma) {
+    if (n_t > 0) {
     // ------------------------------------------------------------ MMA issue (converged warp)
     constexpr uint32_t idesc_score = instr_desc_f16(kTile, kTile, FP16, false);
     constexpr uint32_t idesc_acc = instr_desc_f16(kTile, D, FP16, true);
@@ -734,6 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_elect(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0);
     }
+    }
   } else {
     // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
     const int wg = warp / 4;                  // column half of every score tile
@@ -748,15 +900,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < n_t; ++t) {
       const int first_col = t * kTile + 64 * wg;  // first key of this warpgroup's half
       const uint32_t t_s = tmem + lane_base + C::kColS0 + 128 * (t & 1) + 64 * wg;
-      const bool masked = (causal && t == tile) || (t + 1) * kTile > N;
+      // masked: the causal boundary cuts the tile (its last key is not seen by
+      // the tile's first query), or the keys run out
+      const bool masked = (causal && t * kTile + kTile - 1 > tile * kTile + sq.delta) || (t + 1) * kTile > sq.nk;
       ok = warp_wait_bar(bar(C::kBarSFull + (t & 1)), static_cast<uint32_t>((t >> 1) & 1), wc);
       if (!ok) break;
       tc_fence_after();
       float p[64];
       if (masked) {
-        phase_a<FP16, false, true, false>(t_s, c, nl_row, nullptr, first_col, r_abs, N, causal, p);
+        phase_a<FP16, false, true, false>(t_s, c, nl_row, nullptr, first_col, r_abs, sq.nk, causal, sq.delta, p);
       } else {
-        phase_a<FP16, false, false, false>(t_s, c, nl_row, nullptr, first_col, r_abs, N, causal, p);
+        phase_a<FP16, false, false, false>(t_s, c, nl_row, nullptr, first_col, r_abs, sq.nk, causal, sq.delta, p);
       }
       ok = warp_wait_bar(bar(C::kBarDPFull), static_cast<uint32_t>(t & 1), wc);
       if (!ok) break;
@@ -767,12 +921,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(C::kBarB + wg));
     }
-    if (ok) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
+    if (ok && n_t > 0) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
     if (ok) {
       tc_fence_after();
-      // warpgroup h writes dQ columns h D/2 .. (scaled)
-      const bool row_valid = r_abs < N && index_ok(static_cast<int64_t>(b) * prm.H + h < prm.BH && h < prm.H);
-      uint16_t* dst_row = prm.out0 + ((static_cast<int64_t>(b) * N + r_abs) * prm.H + h) * D + wg * (D / 2);
+      // warpgroup h writes dQ columns h D/2 .. (scaled); a tile whose queries
+      // see no key at all gets 0
+      const bool row_valid =
+          r_abs < sq.nq && index_ok(static_cast<int64_t>(sq.q0) + r_abs < prm.total_q && h < prm.Hq);
+      uint16_t* dst_row = prm.out0 + ((static_cast<int64_t>(sq.q0) + r_abs) * prm.Hq + h) * D + wg * (D / 2);
       const uint32_t acc = tmem + lane_base + C::kColAcc + wg * (D / 2);
 #pragma unroll
       for (int q = 0; q < D / 64; ++q) {
@@ -782,7 +938,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * prm.scale, __uint_as_float(a[2 * k + 1]) * prm.scale);
+          pk[k] = n_t > 0 ? pack2<FP16>(__uint_as_float(a[2 * k]) * prm.scale, __uint_as_float(a[2 * k + 1]) * prm.scale)
+                          : 0u;
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
 #pragma unroll

@@ -335,10 +335,10 @@ Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, in
 // ---------------------------------------------------------------- backward
 
 // Workspace of the backward: D_i = dO_i . O_i, then LSE_i log2(e), each fp32
-// [B*H, Npad] with Npad = N rounded up to whole 128-row tiles, 256-byte aligned.
-size_t bwd_ws_bytes(int64_t B, int64_t N, int64_t H) {
-  const int64_t npad = (N + kTile - 1) / kTile * kTile;
-  return 2 * align256(static_cast<size_t>(B * H * npad) * 4);
+// [B*Hq, Npad] with Npad = Nq rounded up to whole 128-row tiles, 256-byte aligned.
+size_t bwd_ws_bytes(int64_t B, int64_t Nq, int64_t Hq) {
+  const int64_t npad = (Nq + kTile - 1) / kTile * kTile;
+  return 2 * align256(static_cast<size_t>(B * Hq * npad) * 4);
 }
 
 template <int D, bool FP16, bool KV_SIDE>
@@ -359,6 +359,7 @@ fa_status bwd_launch(int dev, const CUtensorMap& x1, const CUtensorMap& x2, cons
       g_devices[dev].configured |= bit;
     }
   }
+  if (grid == 0) return FA_OK;
   kernel<<<static_cast<unsigned>(grid), bwd::kThreads, kSmem, stream>>>(x1, x2, y1, y2, prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -368,39 +369,80 @@ fa_status bwd_launch(int dev, const CUtensorMap& x1, const CUtensorMap& x2, cons
   return FA_OK;
 }
 
+// Backward shape: q, o, dout, dq [B, Nq, Hq, D]; k, v, dk, dv [B, Nk, Hkv, D]
+// (dense: cu_q == nullptr), or packed sequences [total_q, Hq, D] and
+// [total_k, Hkv, D] with device offsets cu_q, cu_k (Nq, Nk: upper bounds of
+// the sequences' lengths).
+struct BwdShape {
+  const int* cu_q;
+  const int* cu_k;
+  int64_t B, Nq, Nk, Hq, Hkv, total_q, total_k;
+};
+
+BwdShape dense_bwd_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv) {
+  return BwdShape{nullptr, nullptr, B, Nq, Nk, Hq, Hkv, B * Nq, B * Nk};
+}
+
 template <int D, bool FP16>
 fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const void* o, const float* lse,
-                  const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, float scale,
-                  int causal, void* workspace, cudaStream_t stream) {
-  const int64_t n_tiles = (N + kTile - 1) / kTile;
-  const int64_t npad = n_tiles * kTile;
-  const int64_t BH = B * H;
+                  const void* dout, void* dq, void* dk, void* dv, const BwdShape& sh, float scale, int causal,
+                  void* workspace, cudaStream_t stream) {
+  const int64_t B = sh.B, Nq = sh.Nq, Nk = sh.Nk, Hq = sh.Hq, Hkv = sh.Hkv;
+  const int64_t tq_rows = sh.total_q, tk_rows = sh.total_k;
+  const int64_t n_qt = (Nq + kTile - 1) / kTile;
+  const int64_t n_kt = (Nk + kTile - 1) / kTile;
+  const int64_t npad = n_qt * kTile;
+  const int64_t BHq = B * Hq;
   float* ws_d = static_cast<float*>(workspace);
-  float* ws_l = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BH * npad) * 4));
+  float* ws_l = ws_d ? reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BHq * npad) * 4))
+                     : nullptr;
   constexpr int64_t kPrepRows = 256 / (D / 8);  // rows per preprocess block
-  const int64_t real_blocks = (B * N * H + kPrepRows - 1) / kPrepRows;
-  const int64_t pad_blocks = (BH * (npad - N) + 255) / 256;
-  bwd::fa_bwd_prep_kernel<D, FP16><<<static_cast<unsigned>(real_blocks + pad_blocks), 256, 0, stream>>>(
-      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(B),
-      static_cast<int>(N), static_cast<int>(H), static_cast<int>(npad), static_cast<unsigned>(real_blocks));
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error("backward preprocess launch", e);
-    return FA_ERR_CUDA;
+  const int64_t real_blocks = (tq_rows * Hq + kPrepRows - 1) / kPrepRows;
+  const int64_t pad_blocks = sh.cu_q ? (BHq * npad + 255) / 256 : (BHq * (npad - Nq) + 255) / 256;
+  if (real_blocks + pad_blocks > 0) {
+    const unsigned grid = static_cast<unsigned>(real_blocks + pad_blocks);
+    if (sh.cu_q) {
+      bwd::fa_bwd_prep_varlen_kernel<D, FP16><<<grid, 256, 0, stream>>>(
+          static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, sh.cu_q,
+          static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(tq_rows), static_cast<int>(npad),
+          static_cast<unsigned>(real_blocks));
+    } else {
+      bwd::fa_bwd_prep_kernel<D, FP16><<<grid, 256, 0, stream>>>(
+          static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(B),
+          static_cast<int>(Nq), static_cast<int>(Hq), static_cast<int>(npad), static_cast<unsigned>(real_blocks));
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_error("backward preprocess launch", e);
+      return FA_ERR_CUDA;
+    }
   }
   const bool fp16 = FP16;
+  // With no queries (or no keys) nothing is ever loaded from that side; its
+  // maps only need a valid, aligned base.
+  const void* qb = tq_rows > 0 ? q : k;
+  const void* dob = tq_rows > 0 ? dout : k;
+  const void* kb = tk_rows > 0 ? k : q;
+  const void* vb = tk_rows > 0 ? v : q;
   CUtensorMap tq, tk, tv, tdo;
-  if (make_tmap(&tq, q, B * N, H, D, fp16) != FA_OK || make_tmap(&tk, k, B * N, H, D, fp16) != FA_OK ||
-      make_tmap(&tv, v, B * N, H, D, fp16) != FA_OK || make_tmap(&tdo, dout, B * N, H, D, fp16) != FA_OK)
+  if (make_tmap(&tq, qb, tq_rows > 0 ? tq_rows : 1, tq_rows > 0 ? Hq : 1, D, fp16) != FA_OK ||
+      make_tmap(&tdo, dob, tq_rows > 0 ? tq_rows : 1, tq_rows > 0 ? Hq : 1, D, fp16) != FA_OK ||
+      make_tmap(&tk, kb, tk_rows > 0 ? tk_rows : 1, tk_rows > 0 ? Hkv : 1, D, fp16) != FA_OK ||
+      make_tmap(&tv, vb, tk_rows > 0 ? tk_rows : 1, tk_rows > 0 ? Hkv : 1, D, fp16) != FA_OK)
     return FA_ERR_CUDA;
   bwd::Params prm;
+  prm.cu_q = sh.cu_q;
+  prm.cu_k = sh.cu_k;
+  prm.total_q = static_cast<int>(tq_rows);
+  prm.total_k = static_cast<int>(tk_rows);
   prm.ws_d = ws_d;
   prm.ws_l = ws_l;
-  prm.N = static_cast<int>(N);
-  prm.H = static_cast<int>(H);
-  prm.BH = static_cast<int>(BH);
+  prm.Nq = static_cast<int>(Nq);
+  prm.Nk = static_cast<int>(Nk);
+  prm.Hq = static_cast<int>(Hq);
+  prm.Hkv = static_cast<int>(Hkv);
+  prm.G = static_cast<int>(Hq / Hkv);
   prm.Npad = static_cast<int>(npad);
-  prm.n_tiles = static_cast<int>(n_tiles);
   // same base-2 factor as the forward (see launch)
   float c = scale * 1.44269504088896340736f;
   if (std::fabs(c) < FLT_MIN) c = std::signbit(c) ? -FLT_MIN : FLT_MIN;
@@ -408,39 +450,56 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
   prm.scale = scale;
   prm.causal = causal ? 1 : 0;
   prm.wait_limit_ns = kDefaultWaitLimitNs;
-  const int64_t grid = n_tiles * BH;
+  // query side: one CTA per (query tile, b, query head)
   prm.out0 = static_cast<uint16_t*>(dq);
   prm.out1 = nullptr;
-  fa_status st = bwd_launch<D, FP16, false>(dev, tq, tdo, tk, tv, prm, grid, stream);
+  prm.BH = static_cast<int>(BHq);
+  prm.n_tiles = static_cast<int>(n_qt);
+  fa_status st = bwd_launch<D, FP16, false>(dev, tq, tdo, tk, tv, prm, n_qt * BHq, stream);
   if (st != FA_OK) return st;
+  // key side: one CTA per (key tile, b, K/V head)
   prm.out0 = static_cast<uint16_t*>(dk);
   prm.out1 = static_cast<uint16_t*>(dv);
-  st = bwd_launch<D, FP16, true>(dev, tk, tv, tq, tdo, prm, grid, stream);
+  prm.BH = static_cast<int>(B * Hkv);
+  prm.n_tiles = static_cast<int>(n_kt);
+  st = bwd_launch<D, FP16, true>(dev, tk, tv, tq, tdo, prm, n_kt * B * Hkv, stream);
   if (st != FA_OK) return st;
   if (debug_enabled())
-    std::fprintf(stderr, "[fa] bwd D=%d %s B=%lld N=%lld H=%lld causal=%d grid=2x%lld\n", D, FP16 ? "fp16" : "bf16",
-                 (long long)B, (long long)N, (long long)H, causal, (long long)grid);
+    std::fprintf(stderr, "[fa] bwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d grid=%lld+%lld\n", D,
+                 FP16 ? "fp16" : "bf16", (long long)B, (long long)Nq, (long long)Nk, (long long)Hq, (long long)Hkv,
+                 sh.cu_q ? "packed" : "dense", causal, (long long)(n_qt * BHq), (long long)(n_kt * B * Hkv));
   return FA_OK;
 }
 
 fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                   void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
+                   void* dq, void* dk, void* dv, const BwdShape& sh, int64_t D, float scale, int causal,
                    fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  if (B < 0 || N < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  const int64_t B = sh.B, Nq = sh.Nq, Nk = sh.Nk, Hq = sh.Hq, Hkv = sh.Hkv;
+  const int64_t tq_rows = sh.total_q, tk_rows = sh.total_k;
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq < 0 || Hkv < 0 || tq_rows < 0 || tk_rows < 0) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (Hq > 0 && (Hkv < 1 || Hq % Hkv != 0)) return FA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (B == 0 || N == 0 || H == 0) return FA_OK;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  if (B * N > INT32_MAX - 2 * kTile || H > INT32_MAX || B * H > INT32_MAX / ((N + kTile - 1) / kTile + 1))
+  if (B == 0 || Hq == 0 || (tq_rows == 0 && tk_rows == 0)) return FA_OK;
+  if (tq_rows > 0 && (!q || !o || !lse || !dout || !dq)) return FA_ERR_INVALID_ARG;
+  if (tk_rows > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if (sh.cu_q && !sh.cu_k) return FA_ERR_INVALID_ARG;
+  const int64_t n_qt = (Nq + kTile - 1) / kTile, n_kt = (Nk + kTile - 1) / kTile;
+  if (tq_rows > INT32_MAX - 2 * kTile || tk_rows > INT32_MAX - 2 * kTile || Nq > INT32_MAX - 2 * kTile ||
+      Nk > INT32_MAX - 2 * kTile || Hq > INT32_MAX || B * Hq > INT32_MAX / (n_qt + 1) ||
+      B * Hkv > INT32_MAX / (n_kt + 1))
     return FA_ERR_UNSUPPORTED;
-  if (static_cast<double>(B) * N * H * D * 2 >= 1099511627776.0) return FA_ERR_UNSUPPORTED;
-  // preprocess grid: B N H / 16 row blocks plus B H (Npad - N) / 256 pad blocks stay below 2^31
-  if (B * H * ((N + kTile - 1) / kTile * kTile) / 15 >= INT32_MAX) return FA_ERR_UNSUPPORTED;
-  if (workspace_bytes < bwd_ws_bytes(B, N, H)) return FA_ERR_INVALID_ARG;
-  for (const void* p : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
-                        static_cast<const void*>(dv), static_cast<const void*>(lse)})
-    if (!aligned16(p)) return FA_ERR_MISALIGNED;
+  if (static_cast<double>(tq_rows) * Hq * D * 2 >= 1099511627776.0 ||
+      static_cast<double>(tk_rows) * Hkv * D * 2 >= 1099511627776.0)
+    return FA_ERR_UNSUPPORTED;
+  // preprocess grid: total_q Hq / 16 row blocks plus at most B Hq Npad / 256 pad blocks stay below 2^31
+  if ((tq_rows * Hq + B * Hq * (n_qt * kTile)) / 15 >= INT32_MAX) return FA_ERR_UNSUPPORTED;
+  const size_t need = bwd_ws_bytes(B, Nq, Hq);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv), static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
   int dev = 0;
   fa_status st = check_device(&dev);
@@ -450,10 +509,10 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool fp16 = dtype == FA_FP16;
   if (D == 128)
-    return fp16 ? bwd_run<128, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s)
-                : bwd_run<128, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s);
-  return fp16 ? bwd_run<64, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s)
-              : bwd_run<64, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, B, N, H, scale, causal, workspace, s);
+    return fp16 ? bwd_run<128, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, sh, scale, causal, workspace, s)
+                : bwd_run<128, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, sh, scale, causal, workspace, s);
+  return fp16 ? bwd_run<64, true>(dev, q, k, v, o, lse, dout, dq, dk, dv, sh, scale, causal, workspace, s)
+              : bwd_run<64, false>(dev, q, k, v, o, lse, dout, dq, dk, dv, sh, scale, causal, workspace, s);
 }
 
 }  // namespace
@@ -700,9 +759,40 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
                  fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
   try {
-    return fa::finish(fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H, D, scale, causal, dtype, workspace,
-                                    workspace_bytes, stream),
+    if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    return fa::finish(fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, fa::dense_bwd_shape(B, N, N, H, H), D, scale,
+                                    causal, dtype, workspace, workspace_bytes, stream),
                       stream, "fa_bwd");
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv,
+                     int64_t D, float scale, int causal, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                     fa_stream_t stream) {
+  try {
+    if (B < 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    return fa::finish(fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, fa::dense_bwd_shape(B, Nq, Nk, Hq, Hkv), D,
+                                    scale, causal, dtype, workspace, workspace_bytes, stream),
+                      stream, "fa_bwd_gqa");
+  } catch (...) {
+    return FA_ERR_CUDA;
+  }
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int64_t B, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                        int64_t total_q, int64_t total_k, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal,
+                        fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  try {
+    if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+    const fa::BwdShape sh{cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, total_q, total_k};
+    return fa::finish(fa::bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, sh, D, scale, causal, dtype, workspace,
+                                    workspace_bytes, stream),
+                      stream, "fa_bwd_varlen");
   } catch (...) {
     return FA_ERR_CUDA;
   }

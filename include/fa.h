@@ -228,6 +228,7 @@ fa_status fa_status_sync(fa_stream_t stream);
 /*
  * fa_bwd_workspace_size - bytes of device workspace fa_bwd needs for these
  * sizes: two fp32 arrays [B*H, ceil(N/128)*128], each rounded up to 256 bytes.
+ * For fa_bwd_gqa pass the query side's sizes (B, Nq, Hq).
  * Returns FA_ERR_INVALID_ARG for a NULL output or a negative size.
  */
 fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspace_bytes);
@@ -267,6 +268,59 @@ fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspa
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                  void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int causal,
                  fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_bwd_gqa - fa_bwd generalised like fa_fwd_gqa: grouped-query heads and
+ * queries and keys of different lengths (cross-attention), the gradients of
+ * fa_fwd_gqa's output; fa_bwd(..., N, H, ...) is fa_bwd_gqa(..., Nq = Nk = N,
+ * Hq = Hkv = H, ...).
+ *
+ *   q, o, dout, dq : [B, Nq, Hq,  D]        k, v, dk, dv : [B, Nk, Hkv, D]
+ *   lse            : float32 [B, Hq, Nq], as fa_fwd_gqa returned it
+ *   Hq % Hkv == 0; query head h reads key/value head h / (Hq / Hkv), so the
+ *     gradient of a key/value head is the sum over the Hq / Hkv query heads
+ *     that read it (grouped-query attention: llmtrend.com FlashAttention page,
+ *     Mistral case; separate query and key lengths: the same page's
+ *     limitations section, cross-attention). The sum is taken inside one CTA
+ *     in a fixed order: results stay deterministic, with no atomics.
+ *   causal : the bottom-right aligned mask of fa_fwd_gqa (key j visible to
+ *            query i iff j <= i + Nk - Nq). A query that sees no key gets
+ *            dQ = 0; a key that no query sees gets dK = dV = 0.
+ *   workspace : at least fa_bwd_workspace_size(B, Nq, Hq) bytes (may be NULL
+ *               when that is 0, i.e. Nq == 0).
+ * Errors and asynchrony as fa_bwd; Hkv < 1 or Hq % Hkv != 0 -> FA_ERR_INVALID_ARG.
+ * B == 0, Hq == 0, or Nq == Nk == 0 returns FA_OK without launching; Nq == 0
+ * with Nk > 0 writes dk = dv = 0, Nk == 0 with Nq > 0 writes dq = 0.
+ */
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv,
+                     int64_t D, float scale, int causal, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                     fa_stream_t stream);
+
+/*
+ * fa_bwd_varlen - the backward of fa_fwd_varlen: B sequences of different
+ * lengths packed without padding (the padding-free form of the pages'
+ * padding mask, jsqmd.com page, usage notes), grouped-query heads, the
+ * bottom-right causal mask per sequence.
+ *
+ *   q, o, dout, dq : [total_q, Hq,  D]; sequence b owns query rows
+ *                    cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *   k, v, dk, dv   : [total_k, Hkv, D]; key rows cu_seqlens_k[b] ..
+ *   lse            : float32 [Hq, total_q], as fa_fwd_varlen returned it
+ *   cu_seqlens_q/k : int32 DEVICE arrays of B+1 non-decreasing offsets
+ *   max_seqlen_q/k : >= every query / key length (size the grids)
+ *   workspace      : at least fa_bwd_workspace_size(B, max_seqlen_q, Hq) bytes
+ * Gradients, masks, grouped heads and determinism as fa_bwd_gqa, per
+ * sequence. As in fa_fwd_varlen the kernels check the offsets: a sequence
+ * whose offsets are inconsistent (decreasing, beyond the totals, or longer
+ * than the maxima) is skipped, its gradients are left untouched, and
+ * fa_status_sync reports FA_ERR_INVALID_ARG.
+ */
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int64_t B, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                        int64_t total_q, int64_t total_k, int64_t Hq, int64_t Hkv, int64_t D, float scale, int causal,
+                        fa_dtype dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_fwd_debug - fa_fwd with two test hooks (same arguments first).
