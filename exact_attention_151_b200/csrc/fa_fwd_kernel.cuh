@@ -86,7 +86,9 @@ constexpr uint32_t kLaunchRegs = 168;
 constexpr uint32_t kSoftmaxRegs = 208;
 constexpr uint32_t kControlRegs = 88;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs, "register split");
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The running max is raised only when a tile's max exceeds it by more than
+// this (log2 units), so P = 2^(x - m) <= 2^15 stays inside fp16's range.
+constexpr float kRescaleThreshold = 15.0f;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kMaxPolls = 1u << 28;
@@ -172,11 +174,6 @@ __device__ __forceinline__ bool split_p_tile(int qt, int j, int causal, int delt
   return j == 0 && (causal ? (qt * kTile <= kTile - 1 - delta) : (nk <= kTile));
 }
 
-// Pairs of score columns whose exp2 runs on the FMA pipe instead of the
-// MUFU unit (every fourth pair): the two softmax warpgroups share each SM
-// sub-partition's exp unit, which the tensor cores otherwise outrun.
-__device__ __forceinline__ constexpr bool emulated_pair(int pair) { return (pair & 3) == 3; }
-
 // Max (MAX) or min of one row of 128 scores: three-input max in four
 // independent chains.
 template <bool MAX>
@@ -216,12 +213,7 @@ __device__ __forceinline__ float softmax_exp_half(const float (&s)[kTile], float
     for (int q = 0; q < 16; ++q) {
       const int pr = HALF * 32 + chunk * 16 + q;  // pair index in the row
       const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
-      float2 p;
-      if (emulated_pair(pr)) {
-        p = exp2_poly2(x);
-      } else {
-        p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-      }
+      const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       if (q & 1) {
         acc1 = fadd2(acc1, p);
       } else {
@@ -238,6 +230,31 @@ __device__ __forceinline__ float softmax_exp_half(const float (&s)[kTile], float
   }
   const float2 acc = fadd2(acc0, acc1);
   return acc.x + acc.y;
+}
+
+// Chunk CH (0..3) of one row of one score tile (keys 32 CH .. 32 CH + 31, i.e.
+// pairs 16 CH .. 16 CH + 15): p = 2^(s * c - m) packed to 16-bit pairs into
+// pk (the caller stores them to TMEM columns 16 CH ..); returns the fp32 sum
+// of p as two partial sums. Nothing is stored, so the caller decides where the
+// TMEM stores and hand-offs go.
+template <bool FP16, int CH>
+__device__ __forceinline__ float2 softmax_exp_chunk(const float (&s)[kTile], float c, float m, uint32_t (&pk)[16]) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int pr = CH * 16 + q;  // pair index in the row
+    const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
+    const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    if (q & 1) {
+      acc1 = fadd2(acc1, p);
+    } else {
+      acc0 = fadd2(acc0, p);
+    }
+    pk[q] = pack2<FP16>(p.x, p.y);
+  }
+  return fadd2(acc0, acc1);
 }
 
 // O row *= alpha in TMEM (warp-collective; D columns from o_col).
@@ -650,6 +667,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // packed heads: a warp whose 32 rows are all past the G Nq real ones only
     // keeps the hand-offs (its rows' O is never stored)
     const bool warp_idle = pg && quarter * 32 >= pg * nq;
+    // Speculate (exponentials before the tile max) until a tile's max outgrows
+    // the threshold once: rows whose max keeps growing (very large logits)
+    // then take the max-first path for the rest of the item. Warp-uniform.
+    bool speculate = true;
     for (int j = 0; j <= last; ++j) {
       ok = warp_wait_bar(bar(C::kBarSFull + wg), static_cast<uint32_t>(j & 1), wc);
       if (!ok) break;
@@ -660,6 +681,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(C::kBarPFull + 2 * wg + 1));
         continue;
       }
+      const int kbase = (jb + j) * kTile;
+      // masking is needed when some row of the tile sees only part of it: the
+      // tile runs past the keys, or past the first row's last visible key
+      const bool masked = kbase + kTile > nk || (causal && kbase + kTile - 1 > q_min(qt) + delta);
+      // last visible column of this row in this tile (may be < 0: none)
+      const int lastcol = (causal ? min(nk - 1, qi + delta) : (nk - 1)) - kbase;
+      if (j > 0 && speculate) {
+        // Fast path for every tile after the first: the running max m_used is
+        // known, and as long as this tile's max exceeds it by at most
+        // kRescaleThreshold, P = 2^(x - m_used) is exactly what the lazy
+        // rescale uses. So the first half's exponentials start at once and the
+        // tile max (an independent chain) runs alongside them. The first
+        // half's P stays in registers until the max is checked: if the max
+        // grew past the threshold (rare after the first tile) nothing has been
+        // written, and the tile is redone below from the scores still in TMEM.
+        float sf[kTile];
+        {
+          uint32_t r[4][32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld32(s_col + q * 32, r[q]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < kTile; ++k) sf[k] = __uint_as_float(r[k / 32][k % 32]);
+        }
+        if (masked) {
+#pragma unroll
+          for (int k = 0; k < kTile; ++k) sf[k] = (k <= lastcol) ? sf[k] : fill;
+        }
+        const float m_raw = c_pos ? row_reduce<true>(sf) : row_reduce<false>(sf);
+        uint32_t pk0[16], pk1[16];
+        float2 acc = softmax_exp_chunk<FP16, 0>(sf, c, m_used, pk0);
+        acc = fadd2(acc, softmax_exp_chunk<FP16, 1>(sf, c, m_used, pk1));
+        if (!__any_sync(0xffffffffu, m_raw * c > m_used + kRescaleThreshold)) {
+          tmem_st16(s_col, pk0);
+          tmem_st16(s_col + 16, pk1);
+          // the second half's first chunk is computed while those stores complete
+          uint32_t pk2[16];
+          float2 acc2 = softmax_exp_chunk<FP16, 2>(sf, c, m_used, pk2);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::kBarPFull + 2 * wg));
+          tmem_st16(s_col + 32, pk2);
+          acc2 = fadd2(acc2, softmax_exp_chunk<FP16, 3>(sf, c, m_used, pk2));
+          tmem_st16(s_col + 48, pk2);
+          const float2 tot = fadd2(acc, acc2);
+          l_sum += tot.x + tot.y;
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::kBarPFull + 2 * wg + 1));
+          continue;
+        }
+        speculate = false;  // the max grew: this warp's later tiles start with the max
+      }
+      // First tile of the range (the running max starts here), a tile whose
+      // max grew past the threshold, or any tile after one: the tile max
+      // comes first.
       float s[kTile];
       {
         uint32_t r[4][32];
@@ -669,12 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kTile; ++k) s[k] = __uint_as_float(r[k / 32][k % 32]);
       }
-      const int kbase = (jb + j) * kTile;
-      // masking is needed when some row of the tile sees only part of it: the
-      // tile runs past the keys, or past the first row's last visible key
-      if (kbase + kTile > nk || (causal && kbase + kTile - 1 > q_min(qt) + delta)) {
-        // last visible column of this row in this tile (may be < 0: none)
-        const int lastcol = (causal ? min(nk - 1, qi + delta) : (nk - 1)) - kbase;
+      if (masked) {
 #pragma unroll
         for (int k = 0; k < kTile; ++k) s[k] = (k <= lastcol) ? s[k] : fill;
       }
