@@ -674,6 +674,8 @@ def run_forward(args, w, dev, world, rank):
         achieved = kernel_flops / (avg_launch_ms * 1e-3) / 1e12
         traffic, traffic_how = recorded_traffic(w.name)
         intensity = w.flops / w.min_hbm_bytes
+        # the kernel's roofline: tensor-bound above the ridge of the measured peaks
+        ridge = peak * 1e12 / (measured_hbm() * 1e9)
         cfg = workload_config(w)
         if shard:
             cfg["parallelism"] = (f"shard over {'batch' if shard[0].axis == 0 else 'heads'} on {world} rank(s) "
@@ -690,7 +692,7 @@ def run_forward(args, w, dev, world, rank):
                           "frac_of_sustained_peak": achieved / peak_sus,
                           "algorithmic_bytes": w.min_hbm_bytes,
                           "traffic_source": traffic_how}
-                         if intensity >= 300 else
+                         if intensity >= ridge else
                          {"bound": "hbm", "achieved": w.min_hbm_bytes / (avg_launch_ms * 1e-3) / 1e9,
                           "peak": measured_hbm(), "unit": "GB/s",
                           "frac": w.min_hbm_bytes / (avg_launch_ms * 1e-3) / 1e9 / measured_hbm(),

@@ -200,7 +200,18 @@ __device__ __forceinline__ float row_reduce(const float (&s)[kTile]) {
 // TMEM columns 32h .. 32h+31 of S_i in two 16-column chunks; with SPLIT also
 // the rounding residual p - p16 to columns 64 + 32h .. Returns the fp32 sum
 // of p. Each score register dies once its pair is packed.
-template <bool FP16, bool SPLIT, int HALF>
+// Pairs of score columns whose exp2 runs on the FMA pipe (a Cody-Waite
+// reduction and a polynomial) instead of the MUFU unit. At D = 64 a score
+// tile carries half the tensor work of D = 128 for the same number of
+// exponentials, so the exp unit alone would outlast the tensor cores: every
+// fourth pair goes to the FMA pipe there. At D = 128 the exponentials fit the
+// MUFU unit and the polynomial's extra instructions cost more than they save.
+template <int D>
+__device__ __forceinline__ constexpr bool fma_exp_pair(int pair) {
+  return D == 64 && (pair & 3) == 3;
+}
+
+template <bool FP16, bool SPLIT, int HALF, int D>
 __device__ __forceinline__ float softmax_exp_half(const float (&s)[kTile], float c, float m, uint32_t s_col) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m, -m);
@@ -213,7 +224,7 @@ __device__ __forceinline__ float softmax_exp_half(const float (&s)[kTile], float
     for (int q = 0; q < 16; ++q) {
       const int pr = HALF * 32 + chunk * 16 + q;  // pair index in the row
       const float2 x = ffma2(make_float2(s[2 * pr], s[2 * pr + 1]), c2, nm2);
-      const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 p = fma_exp_pair<D>(pr) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
       if (q & 1) {
         acc1 = fadd2(acc1, p);
       } else {
@@ -667,10 +678,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // packed heads: a warp whose 32 rows are all past the G Nq real ones only
     // keeps the hand-offs (its rows' O is never stored)
     const bool warp_idle = pg && quarter * 32 >= pg * nq;
-    // Speculate (exponentials before the tile max) until a tile's max outgrows
+    // Speculate (exponentials before the tile max; D = 128 only: at D = 64 the
+    // exp unit, not the max chain, bounds a tile) until a tile's max outgrows
     // the threshold once: rows whose max keeps growing (very large logits)
     // then take the max-first path for the rest of the item. Warp-uniform.
-    bool speculate = true;
+    bool speculate = D == 128;
     for (int j = 0; j <= last; ++j) {
       ok = warp_wait_bar(bar(C::kBarSFull + wg), static_cast<uint32_t>(j & 1), wc);
       if (!ok) break;
@@ -768,17 +780,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // halves (keys 0-63, 64-127) so the PV MMA can start on the first.
       float psum;
       if (split_p_tile(qt, jb + j, causal, delta, nk)) {
-        psum = softmax_exp_half<FP16, true, 0>(s, c, m_used, s_col);
+        psum = softmax_exp_half<FP16, true, 0, D>(s, c, m_used, s_col);
       } else {
-        psum = softmax_exp_half<FP16, false, 0>(s, c, m_used, s_col);
+        psum = softmax_exp_half<FP16, false, 0, D>(s, c, m_used, s_col);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + 2 * wg));
       if (split_p_tile(qt, jb + j, causal, delta, nk)) {
-        psum += softmax_exp_half<FP16, true, 1>(s, c, m_used, s_col);
+        psum += softmax_exp_half<FP16, true, 1, D>(s, c, m_used, s_col);
       } else {
-        psum += softmax_exp_half<FP16, false, 1>(s, c, m_used, s_col);
+        psum += softmax_exp_half<FP16, false, 1, D>(s, c, m_used, s_col);
       }
       l_sum += psum;
       tmem_wait_st();
