@@ -10,12 +10,16 @@
 //   fa_bwd_prep_kernel   -D_i and -LSE_i log2(e) into a workspace padded to
 //                        whole 128-row tiles (pad rows: D = 0, LSE = +inf, so
 //                        their weights are exactly 0);
-//   fa_bwd_dq_kernel     one CTA per (128-query tile, b, h): S = Q K^T and
+//   fa_bwd_dq_kernel     work items (128-query tile, b, h): S = Q K^T and
 //                        dP = dO V^T into TMEM, dS = P (dP - D), dQ += dS K
 //                        over the key tiles;
-//   fa_bwd_dkdv_kernel   one CTA per (128-key tile, b, h): S^T = K Q^T and
-//                        dP^T = V dO^T into TMEM, P^T and dS^T, dV += P^T dO
-//                        and dK += dS^T Q over the query tiles.
+//   fa_bwd_dkdv_kernel   work items (128-key tile, b, K/V head): S^T = K Q^T
+//                        and dP^T = V dO^T into TMEM, P^T and dS^T, dV += P^T dO
+//                        and dK += dS^T Q over the query tiles of the group's
+//                        query heads.
+// The two gradient kernels are persistent: one CTA per SM works through the
+// items (scheduling below), and each item's result depends only on the item,
+// not on which CTA computed it.
 //
 // Both are warp-specialised: a TMA loader warp (the tile's two fixed operands
 // once, the streamed ones through rings), an MMA warp (converged, one elected
@@ -42,6 +46,7 @@ constexpr int kThreads = 320;  // warps 0-7: compute warpgroups 0 and 1, 8: MMA,
 constexpr int kMma = 8;        // warp index
 constexpr int kLoad = 9;       // warp index
 constexpr int kGroup = 16;     // heads per scheduling group (causal)
+constexpr int kItemReaders = 9;  // warps that read each work-item slot: the MMA warp and the 8 compute warps
 
 template <int D>
 struct Cfg {
@@ -59,14 +64,18 @@ struct Cfg {
   static constexpr int kBarDPFull = kBarSFull + 1;    // dP (or dP^T) in TMEM
   static constexpr int kBarA = kBarDPFull + 1;        // [2] phase A of warpgroup h done (128 arrivals)
   static constexpr int kBarB = kBarA + 2;             // [2] phase B of warpgroup h done (128 arrivals)
-  static constexpr int kBarDone = kBarB + 2;          // last accumulating MMA finished
+  static constexpr int kBarDone = kBarB + 2;          // last accumulating MMA of an item finished
   static constexpr int kBarDrain = kBarDone + 1;
-  static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kWsOff = kBarOff + 128;        // key side, per stage: -LSE log2(e) and -D of the 128 queries
+  static constexpr int kBarXEmpty = kBarDrain + 1;    // last MMA reading X1, X2 of an item finished
+  static constexpr int kBarAccEmpty = kBarXEmpty + 1; // accumulators read out (256 arrivals)
+  static constexpr int kBarItemFull = kBarAccEmpty + 1;   // [2] work-item slot written
+  static constexpr int kBarItemEmpty = kBarItemFull + 2;  // [2] work-item slot read (kItemReaders arrivals)
+  static constexpr int kNumBars = kBarItemEmpty + 2;
+  static constexpr int kWsOff = kBarOff + 256;        // key side, per stage: -LSE log2(e) and -D of the 128 queries
   static constexpr int kWsBytes = 2 * 128 * 4;
   static constexpr int kMiscOff = kWsOff + kStages * kWsBytes;
-  static_assert(kNumBars * 8 <= 128, "barrier area");
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static_assert(kNumBars * 8 <= 256, "barrier area");
+  static constexpr int kSmemBytes = kMiscOff + 32 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // TMEM columns: S^T, dP^T, accumulators acc0 = dK, acc1 = dV.
   static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
@@ -96,6 +105,9 @@ struct Params {
   float scale;
   int causal;
   unsigned long long wait_limit_ns;
+  int n_items;          // work items of this kernel's grid: BH * n_tiles
+  int* sched;           // work-item counter of this launch (zeroed before it)
+  int wide_stores;      // out0 and out1 are 32-byte aligned: gradient rows leave in 32-byte stores
 };
 
 // One sequence's rows and lengths as a CTA sees them.
@@ -137,9 +149,10 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
                                                           const uint16_t* __restrict__ dout,
                                                           const float* __restrict__ lse, float* __restrict__ ws_d,
                                                           float* __restrict__ ws_l, int B, int N, int H, int Npad,
-                                                          unsigned n_real_blocks) {
+                                                          unsigned n_real_blocks, int* __restrict__ sched) {
   constexpr int kLanes = D / 8;                 // threads per row
   constexpr int kRowsPerBlock = 256 / kLanes;
+  if (blockIdx.x == 0 && threadIdx.x < 2) sched[threadIdx.x] = 0;  // the gradient kernels' work-item counters
   const int64_t n_rows = static_cast<int64_t>(B) * N * H;
   if (blockIdx.x < n_real_blocks) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanes;  // (b N + i) H + h
@@ -192,9 +205,11 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_varlen_kernel(const uint16_t*
                                                                  const float* __restrict__ lse,
                                                                  float* __restrict__ ws_d, float* __restrict__ ws_l,
                                                                  const int* __restrict__ cu_q, int B, int H,
-                                                                 int total_q, int Npad, unsigned n_real_blocks) {
+                                                                 int total_q, int Npad, unsigned n_real_blocks,
+                                                                 int* __restrict__ sched) {
   constexpr int kLanes = D / 8;
   constexpr int kRowsPerBlock = 256 / kLanes;
+  if (blockIdx.x == 0 && threadIdx.x < 2) sched[threadIdx.x] = 0;  // the gradient kernels' work-item counters
   if (blockIdx.x < n_real_blocks) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanes;  // r H + h
     const int sub = threadIdx.x % kLanes;
@@ -335,12 +350,103 @@ __device__ __forceinline__ void phase_b(uint32_t t_dp, uint32_t t_out, float nd_
   }
 }
 
-// Key side: a tile of 128 keys of one K/V head; X1 = K, X2 = V stay in shared
-// memory, and (Q_t, dO_t) stream through a two-stage ring, each stage with the
-// tile's -LSE log2(e) and -D, as items u = (g, t): for each of the G query
-// heads g that read this K/V head, the query tiles t whose queries see some
-// key of the tile. dK and dV accumulate over all items in TMEM (a fixed order,
-// no atomics); out0 = dK, out1 = dV.
+// Persistent scheduling (both gradient kernels). A launch runs one CTA per SM
+// (at most one per work item). A CTA's first item is its block index. With
+// the causal mask every further one comes from the launch's counter (zeroed
+// before the launch), so a CTA that finishes early takes the next item and
+// the lightest items, last in the order, fill the tail; without it items cost
+// the same and a CTA takes every gridDim-th. The loader warp draws the items and hands each
+// to the MMA warp and the compute warps through a two-slot ring in shared
+// memory (-1 once the items run out). The mbarrier phases run on across
+// items, counted by running totals (tiles streamed, items with work), so the
+// next item's fixed operands load and its first score products are issued
+// while the compute warps still write out the current item's gradients.
+
+// Loader warp: item x (or -1) into slot i % 2, once the readers are done with
+// the item that slot held before.
+__device__ __forceinline__ bool item_publish(volatile int* slots, uint32_t full0, uint32_t empty0, int i, int x,
+                                             WaitCtl wc) {
+  const int slot = i & 1;
+  if (i >= 2 && !warp_wait_bar(empty0 + 8 * slot, static_cast<uint32_t>(((i >> 1) & 1) ^ 1), wc)) return false;
+  if ((threadIdx.x & 31) == 0) {
+    slots[slot] = x;
+    mbar_arrive(full0 + 8 * slot);  // release: the slot's value is visible to the waiters
+  }
+  __syncwarp();
+  return true;
+}
+
+// A reading warp: the item in slot i % 2 (-1: no more), or -2 if the CTA is aborting.
+__device__ __forceinline__ int item_take(const volatile int* slots, uint32_t full0, uint32_t empty0, int i,
+                                         WaitCtl wc) {
+  const int slot = i & 1;
+  if (!warp_wait_bar(full0 + 8 * slot, static_cast<uint32_t>((i >> 1) & 1), wc)) return -2;
+  const int x = slots[slot];
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty0 + 8 * slot);
+  return x;
+}
+
+// Loader warp: the CTA's next item after x. Non-causal items all cost the
+// same: a fixed stride keeps the CTAs in step, so CTAs working on the same
+// head ask for the same K/V (or Q/dO) tiles at about the same time and the
+// L2 serves them together. Causal items differ in cost: the counter.
+__device__ __forceinline__ int item_next(int* sched, int x, int causal) {
+  if (!causal) return x + static_cast<int>(gridDim.x);
+  int nx = 0;
+  if ((threadIdx.x & 31) == 0) nx = static_cast<int>(gridDim.x) + atomicAdd(sched, 1);
+  return __shfl_sync(0xffffffffu, nx, 0);
+}
+
+// Key side work item: a tile of 128 keys of one K/V head of one sequence.
+// Causal work per tile is uneven (later key tiles are seen by fewer query
+// tiles): items go in groups of kGroup heads, heaviest tiles first within a
+// group, so the tail holds the short ones and a group's Q/dO stay
+// L2-resident. Non-causal: head-major.
+struct ItemKV {
+  int tile, b, hk;
+  Seq sq;
+  int t_first, per_head;  // query tiles t_first .. n_qt-1 of each of the G query heads see some key of the tile
+  int n_t;                // streamed (query head, query tile) pairs: G * per_head
+  bool skip;              // no work: tile past the sequence's end, or inconsistent packed offsets
+};
+
+__device__ __forceinline__ ItemKV item_kv(const Params& prm, int x) {
+  ItemKV it;
+  int bh;
+  if (prm.causal) {
+    const int per_group = kGroup * prm.n_tiles;
+    const int g = x / per_group;
+    const int r = x % per_group;
+    const int gsize = min(kGroup, prm.BH - g * kGroup);
+    bh = g * kGroup + r % gsize;
+    it.tile = r / gsize;
+  } else {
+    it.tile = x % prm.n_tiles;
+    bh = x / prm.n_tiles;
+  }
+  it.b = bh / prm.Hkv;
+  it.hk = bh % prm.Hkv;
+  it.sq = resolve_seq(prm, it.b);
+  it.skip = !it.sq.ok || it.tile >= it.sq.n_kt;
+  // query tiles that see some key of this tile: from the one holding the first
+  // query i with i + delta >= tile * 128 (causal) to the last
+  it.t_first = 0;
+  if (prm.causal) {
+    const int i0 = it.tile * kTile - it.sq.delta;
+    it.t_first = i0 <= 0 ? 0 : i0 / kTile;
+  }
+  it.per_head = it.skip ? 0 : max(0, it.sq.n_qt - it.t_first);
+  it.n_t = prm.G * it.per_head;
+  return it;
+}
+
+// Key side: items are tiles of 128 keys of one K/V head; X1 = K, X2 = V stay
+// in shared memory for the item, and (Q_t, dO_t) stream through a two-stage
+// ring, each stage with the tile's -LSE log2(e) and -D, as pairs u = (g, t):
+// for each of the G query heads g that read this K/V head, the query tiles t
+// whose queries see some key of the tile. dK and dV accumulate over all pairs
+// in TMEM (a fixed order, no atomics); out0 = dK, out1 = dV.
 // TMEM holds one S^T / dP^T pair beside the two accumulators, so the MMA warp
 // interleaves consecutive tiles, S(0) dP(0) | dV(t) S(t+1) dK(t) dP(t+1) | ...,
 // issuing each accumulating product per half as soon as that half is in TMEM.
@@ -359,45 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto ws_stage = [&](int s) { return sbase + C::kWsOff + s * C::kWsBytes; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  volatile int* item_slots = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int causal = prm.causal;
-  // CTA -> (bh, key tile), bh = b * Hkv + hk. Causal work per tile is uneven
-  // (later key tiles are seen by fewer query tiles): CTAs go in groups of
-  // kGroup heads, heaviest tiles first within a group, so the last wave holds
-  // the short ones and a group's Q/dO stay L2-resident. Non-causal: head-major.
-  int tile, bh;
-  if (causal) {
-    const int per_group = kGroup * prm.n_tiles;
-    const int g = static_cast<int>(blockIdx.x) / per_group;
-    const int r = static_cast<int>(blockIdx.x) % per_group;
-    const int gsize = min(kGroup, prm.BH - g * kGroup);
-    const int level = r / gsize;
-    bh = g * kGroup + r % gsize;
-    tile = level;
-  } else {
-    tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
-    bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
-  }
-  const int b = bh / prm.Hkv, hk = bh % prm.Hkv;
-  const Seq sq = resolve_seq(prm, b);
-  if (!sq.ok) {  // inconsistent packed offsets: report, touch nothing
-    if (threadIdx.x == 0) atomicOr(&g_status_word, 2u);
-    return;
-  }
-  if (tile >= sq.n_kt) return;  // key tile past the end of this sequence
-  // Query tiles that see some key of this tile: from the one holding the
-  // first query i with i + delta >= tile * 128 (causal) to the last.
-  int t_first = 0;
-  if (causal) {
-    const int i0 = tile * kTile - sq.delta;
-    t_first = i0 <= 0 ? 0 : i0 / kTile;
-  }
-  const int per_head = max(0, sq.n_qt - t_first);
-  const int n_t = prm.G * per_head;  // streamed items; item u: query head hk G + u / per_head, tile t_first + u % per_head
-  auto item_head = [&](int u) { return hk * prm.G + u / per_head; };
-  auto item_tile = [&](int u) { return t_first + u % per_head; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarX), 1);
@@ -410,9 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::kBarA + i), 128);
       mbar_init(bar(C::kBarB + i), 128);
+      mbar_init(bar(C::kBarItemFull + i), 1);
+      mbar_init(bar(C::kBarItemEmpty + i), kItemReaders);
     }
     mbar_init(bar(C::kBarDone), 1);
     mbar_init(bar(C::kBarDrain), 1);
+    mbar_init(bar(C::kBarXEmpty), 1);
+    mbar_init(bar(C::kBarAccEmpty), 256);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -425,11 +501,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, prm.wait_limit_ns};
-  const int krow0 = sq.k0;  // first row of this sequence in the [rows, Hkv, D] views
-  const int qrow0 = sq.q0;  // and in the [rows, Hq, D] views
+  const uint32_t full0 = bar(C::kBarItemFull), empty0 = bar(C::kBarItemEmpty);
 
   if (warp == kLoad) {
-    if (n_t > 0) {
     // ------------------------------------------------------------ loader (converged warp)
     if (lane == 0) {
       tma_prefetch_desc(&tm_x1);
@@ -438,41 +512,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_y2);
     }
     __syncwarp();
-    mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
-    for (int hf = 0; hf < C::kHalves; ++hf) {
-      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_x1, hf * 64, hk, krow0 + tile * kTile, bar(C::kBarX));
-      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_x2, hf * 64, hk, krow0 + tile * kTile, bar(C::kBarX));
-    }
-    int issued = 0;
-    for (int t = 0; t < n_t; ++t) {
-      const int s = t % C::kStages;
-      if (t >= C::kStages &&
-          !warp_wait_bar(bar(C::kBarYEmpty + s), static_cast<uint32_t>(((t / C::kStages) & 1) ^ 1), wc))
-        break;
-      const int hq = item_head(t), tq = item_tile(t);
-      const int row = qrow0 + tq * kTile;
-      mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + C::kWsBytes);
-      for (int hf = 0; hf < C::kHalves; ++hf) {
-        tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, hq, row, bar(C::kBarYFull + s));
-        tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, hq, row, bar(C::kBarYFull + s));
+    int x = static_cast<int>(blockIdx.x);
+    int yc = 0, xi = 0;  // (Q, dO) stages and (K, V) pairs loaded so far
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      ok = item_publish(item_slots, full0, empty0, i, x < prm.n_items ? x : -1, wc);
+      if (!ok || x >= prm.n_items) break;
+      const ItemKV it = item_kv(prm, x);
+      if (it.n_t > 0) {
+        // K, V of this item once the previous item's last score products have read theirs
+        if (xi > 0 && !(ok = warp_wait_bar(bar(C::kBarXEmpty), static_cast<uint32_t>((xi - 1) & 1), wc))) break;
+        const int krow = it.sq.k0 + it.tile * kTile;
+        mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_x1, hf * 64, it.hk, krow, bar(C::kBarX));
+          tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_x2, hf * 64, it.hk, krow, bar(C::kBarX));
+        }
+        ++xi;
+        for (int u = 0; u < it.n_t; ++u, ++yc) {
+          const int s = yc % C::kStages;
+          if (yc >= C::kStages &&
+              !(ok = warp_wait_bar(bar(C::kBarYEmpty + s), static_cast<uint32_t>(((yc / C::kStages) & 1) ^ 1), wc)))
+            break;
+          const int hq = it.hk * prm.G + u / it.per_head, tq = it.t_first + u % it.per_head;
+          const int row = it.sq.q0 + tq * kTile;
+          mbar_arrive_expect_tx_elect(bar(C::kBarYFull + s), 2 * C::kTileBytes + C::kWsBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf) {
+            tma_load_3d_elect(y_smem(s, 0) + hf * C::kSlabBytes, &tm_y1, hf * 64, hq, row, bar(C::kBarYFull + s));
+            tma_load_3d_elect(y_smem(s, 1) + hf * C::kSlabBytes, &tm_y2, hf * 64, hq, row, bar(C::kBarYFull + s));
+          }
+          // this query tile's -LSE log2(e) and -D ride with Q_t and dO_t
+          const int64_t ws_row = (static_cast<int64_t>(it.b) * prm.Hq + hq) * prm.Npad + tq * kTile;
+          bulk_load_elect(ws_stage(s), prm.ws_l + ws_row, kTile * 4, bar(C::kBarYFull + s));
+          bulk_load_elect(ws_stage(s) + kTile * 4, prm.ws_d + ws_row, kTile * 4, bar(C::kBarYFull + s));
+        }
+        if (!ok) break;
       }
-      {
-        // this query tile's -LSE log2(e) and -D ride with Q_t and dO_t
-        const int64_t ws_row = (static_cast<int64_t>(b) * prm.Hq + hq) * prm.Npad + tq * kTile;
-        bulk_load_elect(ws_stage(s), prm.ws_l + ws_row, kTile * 4, bar(C::kBarYFull + s));
-        bulk_load_elect(ws_stage(s) + kTile * 4, prm.ws_d + ws_row, kTile * 4, bar(C::kBarYFull + s));
-      }
-      issued = t + 1;
+      x = item_next(prm.sched, x, causal);
     }
     // let the copies this warp issued land before shared memory is released
-    drain_wait(bar(C::kBarX), 0);
-    for (int s = 0; s < C::kStages && s < issued; ++s) {
-      const int tl = s + ((issued - 1 - s) / C::kStages) * C::kStages;
-      drain_wait(bar(C::kBarYFull + s), static_cast<uint32_t>((tl / C::kStages) & 1));
-    }
+    if (xi > 0) drain_wait(bar(C::kBarX), static_cast<uint32_t>((xi - 1) & 1));
+    for (int s = 0; s < C::kStages && s < yc; ++s) {
+      const int last = s + ((yc - 1 - s) / C::kStages) * C::kStages;
+      drain_wait(bar(C::kBarYFull + s), static_cast<uint32_t>((last / C::kStages) & 1));
     }
   } else if (warp == kMma) {
-    if (n_t > 0) {
     // ------------------------------------------------------------ MMA issue (converged warp)
     constexpr uint32_t idesc_score = instr_desc_f16(kTile, kTile, FP16, false);
     constexpr uint32_t idesc_acc = instr_desc_f16(kTile, D, FP16, true);
@@ -501,133 +585,174 @@ __global__ void __launch_bounds__(kThreads, 1)
                      (first && q == 0) ? 0u : 1u);
       }
     };
-    bool ok = warp_wait_bar(bar(C::kBarX), 0, wc) && warp_wait_bar(bar(C::kBarYFull), 0, wc);
-    if (ok) {
+    int yc = 0, tc = 0, xi = 0;  // streamed stages, score tiles and items with work so far
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int x = item_take(item_slots, full0, empty0, i, wc);
+      if (x < 0) {
+        ok = x == -1;
+        break;
+      }
+      const ItemKV it = item_kv(prm, x);
+      const int n = it.n_t;
+      if (n == 0) continue;
+      auto ystage = [&](int t) { return (yc + t) % C::kStages; };
+      auto yphase = [&](int t) { return static_cast<uint32_t>(((yc + t) / C::kStages) & 1); };
+      ok = warp_wait_bar(bar(C::kBarX), static_cast<uint32_t>(xi & 1), wc) &&
+           warp_wait_bar(bar(C::kBarYFull + ystage(0)), yphase(0), wc);
+      if (!ok) break;
       tc_fence_after();
-      issue_score(0, 0, C::kColS);
+      issue_score(0, ystage(0), C::kColS);
       mma_commit_elect(bar(C::kBarSFull));
-      issue_score(1, 0, C::kColDP);
+      issue_score(1, ystage(0), C::kColDP);
       mma_commit_elect(bar(C::kBarDPFull));
-    }
-    for (int t = 0; ok && t < n_t; ++t) {
-      const int s = t % C::kStages;
-      const bool more = t + 1 < n_t;
-      const uint32_t ph = static_cast<uint32_t>(t & 1);
-      const uint32_t ph_next = static_cast<uint32_t>(((t + 1) / C::kStages) & 1);
-      // dV += P^T dO per half as each warpgroup publishes its P^T
-      for (int hf = 0; hf < 2 && ok; ++hf) {
-        ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
-        if (ok) {
-          tc_fence_after();
-          issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, s, hf, t == 0 && hf == 0);
+      if (n == 1) mma_commit_elect(bar(C::kBarXEmpty));  // K, V of this item: last readers issued
+      for (int t = 0; ok && t < n; ++t) {
+        const uint32_t ph = static_cast<uint32_t>((tc + t) & 1);
+        const bool more = t + 1 < n;
+        // dV += P^T dO per half as each warpgroup publishes its P^T; the first
+        // one of an item waits until the previous item's accumulators are read out
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
+          if (ok && t == 0 && hf == 0 && xi > 0)
+            ok = warp_wait_bar(bar(C::kBarAccEmpty), static_cast<uint32_t>((xi - 1) & 1), wc);
+          if (ok) {
+            tc_fence_after();
+            issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, ystage(t), hf, t == 0 && hf == 0);
+          }
         }
-      }
-      if (!ok) break;
-      // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
-      if (more) {
-        ok = warp_wait_bar(bar(C::kBarYFull + (t + 1) % C::kStages), ph_next, wc);
         if (!ok) break;
-        tc_fence_after();
-        issue_score(0, (t + 1) % C::kStages, C::kColS);
-        mma_commit_elect(bar(C::kBarSFull));
-      }
-      // dK += dS^T Q per half
-      for (int hf = 0; hf < 2 && ok; ++hf) {
-        ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
-        if (ok) {
+        // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
+        if (more) {
+          ok = warp_wait_bar(bar(C::kBarYFull + ystage(t + 1)), yphase(t + 1), wc);
+          if (!ok) break;
           tc_fence_after();
-          issue_acc(C::kColAcc0, C::kColDP + 64 * hf, 0, s, hf, t == 0 && hf == 0);
+          issue_score(0, ystage(t + 1), C::kColS);
+          mma_commit_elect(bar(C::kBarSFull));
+        }
+        // dK += dS^T Q per half
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = warp_wait_bar(bar(C::kBarB + hf), ph, wc);
+          if (ok) {
+            tc_fence_after();
+            issue_acc(C::kColAcc0, C::kColDP + 64 * hf, 0, ystage(t), hf, t == 0 && hf == 0);
+          }
+        }
+        if (!ok) break;
+        mma_commit_elect(bar(C::kBarYEmpty + ystage(t)));  // stage t: last reader issued
+        if (more) {
+          // dP of the next tile (after the accumulating products that read this tile's dS)
+          issue_score(1, ystage(t + 1), C::kColDP);
+          mma_commit_elect(bar(C::kBarDPFull));
+          if (t + 1 == n - 1) mma_commit_elect(bar(C::kBarXEmpty));
+        } else {
+          mma_commit_elect(bar(C::kBarDone));
         }
       }
-      if (!ok) break;
-      if (t + C::kStages < n_t) mma_commit_elect(bar(C::kBarYEmpty + s));
-      if (more) {
-        // dP of the next tile (after the accumulating products that read this tile's dS)
-        issue_score(1, (t + 1) % C::kStages, C::kColDP);
-        mma_commit_elect(bar(C::kBarDPFull));
-      } else {
-        mma_commit_elect(bar(C::kBarDone));
-      }
+      yc += n;
+      tc += n;
+      ++xi;
     }
     if (!ok) {
       mma_commit_elect(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0);
-    }
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
     const int wg = warp / 4;                  // column half of every score tile
     const int qd = warp % 4;                  // TMEM lane quadrant
     const int row = qd * 32 + lane;
-    const int r_abs = tile * kTile + row;     // this thread's query (or key) index
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const float c = prm.scale_log2;
     const float nl_row = 0.f, nd_row = 0.f;  // per-column values on this side
     const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
     const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
     const uint32_t t_ds = t_dp;  // dS^T pairs over the first half of this half of dP^T
+    int yc = 0, tc = 0, xi = 0;
     bool ok = true;
-    for (int t = 0; t < n_t; ++t) {
-      const int cbase = item_tile(t) * kTile;  // first query (column) of this item's tile
-      const int first_col = cbase + 64 * wg;
-      const uint32_t ph = static_cast<uint32_t>(t & 1);
-      // key side: this tile's -LSE log2(e) and -D for the warpgroup's 64 query
-      // columns, in the TMA stage (the stage is released after phase B)
-      const int s = t % C::kStages;
-      const float* nl_col = reinterpret_cast<const float*>(smem + C::kWsOff + s * C::kWsBytes) + 64 * wg;
-      const float* nd_col = nl_col + kTile;
-      // masked: the causal boundary cuts the tile (its last key is not seen by
-      // its first query), or the queries run out
-      const bool masked = (causal && tile * kTile + kTile - 1 > cbase + sq.delta) || cbase + kTile > sq.nq;
-      ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((t / C::kStages) & 1), wc);
-      if (!ok) break;
-      ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
-      if (!ok) break;
-      tc_fence_after();
-      float p[64];
-      if (masked) {
-        phase_a<FP16, true, true, true>(t_s, c, nl_row, nl_col, first_col, r_abs, sq.nq, causal, sq.delta, p);
-      } else {
-        phase_a<FP16, true, false, true>(t_s, c, nl_row, nl_col, first_col, r_abs, sq.nq, causal, sq.delta, p);
+    int x = item_take(item_slots, full0, empty0, 0, wc);
+    for (int i = 0; x >= 0; ++i) {
+      const ItemKV it = item_kv(prm, x);
+      if (it.skip) {
+        if (!it.sq.ok && threadIdx.x == 0) atomicOr(&g_status_word, 2u);  // inconsistent packed offsets
+        x = item_take(item_slots, full0, empty0, i + 1, wc);
+        continue;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarA + wg));
-      ok = warp_wait_bar(bar(C::kBarDPFull), ph, wc);
-      if (!ok) break;
-      tc_fence_after();
-      phase_b<FP16, true>(t_dp, t_ds, nd_row, nd_col, p);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarB + wg));
-    }
-    if (ok && n_t > 0) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
-    if (ok) {
-      tc_fence_after();
-      // warpgroup 0 writes dK (scaled), warpgroup 1 dV; no query sees these
-      // keys when there were no items: both are 0
-      const bool row_valid =
-          r_abs < sq.nk && index_ok(static_cast<int64_t>(sq.k0) + r_abs < prm.total_k && hk < prm.Hkv);
-      uint16_t* dst_row = (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(sq.k0) + r_abs) * prm.Hkv + hk) * D;
-      const float mul = wg == 1 ? 1.f : prm.scale;
-      constexpr int kCols = D;
-      const uint32_t acc = tmem + lane_base + (wg == 0 ? C::kColAcc0 : C::kColAcc1);
-      const int col0 = 0;
-#pragma unroll
-      for (int q = 0; q < kCols / 32; ++q) {
-        uint32_t a[32];
-        tmem_ld32(acc + q * 32, a);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pk[k] = n_t > 0 ? pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul) : 0u;
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + col0 + q * 32);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      const int r_abs = it.tile * kTile + row;  // this thread's key
+      for (int t = 0; t < it.n_t; ++t) {
+        const int g = yc + t;
+        const int s = g % C::kStages;
+        const uint32_t ph = static_cast<uint32_t>((tc + t) & 1);
+        const int cbase = (it.t_first + t % it.per_head) * kTile;  // first query (column) of this pair's tile
+        const int first_col = cbase + 64 * wg;
+        // this tile's -LSE log2(e) and -D for the warpgroup's 64 query columns,
+        // in the TMA stage (released after phase B)
+        const float* nl_col = reinterpret_cast<const float*>(smem + C::kWsOff + s * C::kWsBytes) + 64 * wg;
+        const float* nd_col = nl_col + kTile;
+        // masked: the causal boundary cuts the tile (its last key is not seen by
+        // its first query), or the queries run out
+        const bool masked = (causal && it.tile * kTile + kTile - 1 > cbase + it.sq.delta) || cbase + kTile > it.sq.nq;
+        ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((g / C::kStages) & 1), wc);
+        if (!ok) break;
+        ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
+        if (!ok) break;
+        tc_fence_after();
+        float p[64];
+        if (masked) {
+          phase_a<FP16, true, true, true>(t_s, c, nl_row, nl_col, first_col, r_abs, it.sq.nq, causal, it.sq.delta, p);
+        } else {
+          phase_a<FP16, true, false, true>(t_s, c, nl_row, nl_col, first_col, r_abs, it.sq.nq, causal, it.sq.delta, p);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::kBarA + wg));
+        ok = warp_wait_bar(bar(C::kBarDPFull), ph, wc);
+        if (!ok) break;
+        tc_fence_after();
+        phase_b<FP16, true>(t_dp, t_ds, nd_row, nd_col, p);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::kBarB + wg));
       }
+      if (!ok) break;
+      // the next item (published by now: this item's loads have all been issued)
+      const int nx = item_take(item_slots, full0, empty0, i + 1, wc);
+      if (it.n_t > 0 && !(ok = warp_wait_bar(bar(C::kBarDone), static_cast<uint32_t>(xi & 1), wc))) break;
+      // warpgroup 0 writes dK (scaled), warpgroup 1 dV; no query sees these
+      // keys when there were no pairs: both are 0. After the last read of the
+      // accumulator it goes back to the MMA warp (the next item's first dV
+      // waits for that and for this warpgroup's next phase A anyway).
+      const bool row_valid =
+          r_abs < it.sq.nk && index_ok(static_cast<int64_t>(it.sq.k0) + r_abs < prm.total_k && it.hk < prm.Hkv);
+      uint16_t* dst_row =
+          (wg == 1 ? prm.out1 : prm.out0) + ((static_cast<int64_t>(it.sq.k0) + r_abs) * prm.Hkv + it.hk) * D;
+      const float mul = wg == 1 ? 1.f : prm.scale;
+      const uint32_t acc = tmem + lane_base + (wg == 0 ? C::kColAcc0 : C::kColAcc1);
+      if (it.n_t > 0) tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t pk[16];
+        if (it.n_t > 0) {
+          uint32_t a[32];
+          tmem_ld32(acc + q * 32, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * mul, __uint_as_float(a[2 * k + 1]) * mul);
+          if (q == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarAccEmpty));
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        if (row_valid) store_row64(dst_row + q * 32, pk, prm.wide_stores != 0);
+      }
+      yc += it.n_t;
+      tc += it.n_t;
+      if (it.n_t > 0) ++xi;
+      x = nx;
     }
   }
 
@@ -639,12 +764,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Query side with a double-buffered score tile. One CTA per (128-query tile,
-// b, h); Q and dO stay in shared memory, K_t streams through a three-stage
-// ring and V_t through a two-stage ring. TMEM: S(t) in buffer t % 2 (columns
-// 0 and 128), dP at 256, dQ at 384; dS(t) is written back over the first half
-// of each warpgroup's columns of its own S buffer. The MMA warp waits once per
-// streamed tile, for both warpgroups' dS(t), and then issues
+// Query side work item: a tile of 128 queries of one query head of one
+// sequence; causal in groups of kGroup heads with the heaviest (latest) tiles
+// first, non-causal head-major.
+struct ItemQ {
+  int tile, bh, h, hk;
+  Seq sq;
+  int n_t;    // key tiles 0 .. n_t-1 (causal: up to the one holding the last key the tile's last query sees)
+  bool skip;  // no work: tile past the sequence's end, or inconsistent packed offsets
+};
+
+__device__ __forceinline__ ItemQ item_q(const Params& prm, int x) {
+  ItemQ it;
+  if (prm.causal) {
+    const int per_group = kGroup * prm.n_tiles;
+    const int g = x / per_group;
+    const int r = x % per_group;
+    const int gsize = min(kGroup, prm.BH - g * kGroup);
+    it.bh = g * kGroup + r % gsize;
+    it.tile = prm.n_tiles - 1 - r / gsize;
+  } else {
+    it.tile = x % prm.n_tiles;
+    it.bh = x / prm.n_tiles;
+  }
+  it.h = it.bh % prm.Hq;
+  it.hk = it.h / prm.G;  // the K/V head this query head reads
+  it.sq = resolve_seq(prm, it.bh / prm.Hq);
+  it.skip = !it.sq.ok || it.tile >= it.sq.n_qt;
+  it.n_t = it.skip ? 0 : it.sq.n_kt;
+  if (!it.skip && prm.causal) {
+    const int last_key = it.tile * kTile + kTile - 1 + it.sq.delta;
+    it.n_t = last_key < 0 ? 0 : min(it.sq.n_kt, last_key / kTile + 1);
+  }
+  return it;
+}
+
+// Query side with a double-buffered score tile: items are tiles of 128
+// queries of one query head; Q and dO stay in shared memory for the item, K_t
+// streams through a three-stage ring and V_t through a two-stage ring. TMEM:
+// S(t) in buffer t % 2 (columns 0 and 128; t counted across items), dP at 256,
+// dQ at 384; dS(t) is written back over the first half of each warpgroup's
+// columns of its own S buffer. The MMA warp waits once per streamed tile, for
+// both warpgroups' dS(t), and then issues
 //   dP(t+1), dQ(t), S(t+2)
 // back to back, so the score product two tiles ahead is already in TMEM when
 // the warpgroups need it.
@@ -667,12 +828,16 @@ struct CfgQ {
   static constexpr int kBarSFull = kBarVEmpty + kVStages;         // [2] S buffer b holds S(t), t % 2 == b
   static constexpr int kBarDPFull = kBarSFull + 2;
   static constexpr int kBarB = kBarDPFull + 1;                    // [2] warpgroup h wrote dS(t) (128 arrivals)
-  static constexpr int kBarDone = kBarB + 2;
+  static constexpr int kBarDone = kBarB + 2;                      // last dQ product of an item finished
   static constexpr int kBarDrain = kBarDone + 1;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarXEmpty = kBarDrain + 1;                // last MMA reading Q, dO of an item finished
+  static constexpr int kBarAccEmpty = kBarXEmpty + 1;             // dQ accumulator read out (256 arrivals)
+  static constexpr int kBarItemFull = kBarAccEmpty + 1;           // [2] work-item slot written
+  static constexpr int kBarItemEmpty = kBarItemFull + 2;          // [2] work-item slot read (kItemReaders arrivals)
+  static constexpr int kNumBars = kBarItemEmpty + 2;
   static_assert(kNumBars * 8 <= 256, "barrier area");
   static constexpr int kMiscOff = kBarOff + 256;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr int kSmemBytes = kMiscOff + 32 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kColS0 = 0, kColDP = 256, kColAcc = 384;
   static_assert(384 + D <= 512, "TMEM budget");
@@ -693,39 +858,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return sbase + C::kBarOff + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  volatile int* item_slots = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int causal = prm.causal;
-  // CTA -> (bh, query tile), bh = b * Hq + h: causal in groups of kGroup
-  // heads, heaviest (latest) query tiles first; non-causal head-major.
-  int tile, bh;
-  if (causal) {
-    const int per_group = kGroup * prm.n_tiles;
-    const int g = static_cast<int>(blockIdx.x) / per_group;
-    const int r = static_cast<int>(blockIdx.x) % per_group;
-    const int gsize = min(kGroup, prm.BH - g * kGroup);
-    bh = g * kGroup + r % gsize;
-    tile = prm.n_tiles - 1 - r / gsize;
-  } else {
-    tile = static_cast<int>(blockIdx.x) % prm.n_tiles;
-    bh = static_cast<int>(blockIdx.x) / prm.n_tiles;
-  }
-  const int b = bh / prm.Hq, h = bh % prm.Hq;
-  const int hk = h / prm.G;  // the K/V head this query head reads
-  const Seq sq = resolve_seq(prm, b);
-  if (!sq.ok) {  // inconsistent packed offsets: report, touch nothing
-    if (threadIdx.x == 0) atomicOr(&g_status_word, 2u);
-    return;
-  }
-  if (tile >= sq.n_qt) return;  // query tile past the end of this sequence
-  // key tiles 0 .. n_t-1: all of them, or (causal) up to the one holding the
-  // last key the tile's last query sees; none if no query of the tile sees a key
-  int n_t = sq.n_kt;
-  if (causal) {
-    const int last_key = tile * kTile + kTile - 1 + sq.delta;
-    n_t = last_key < 0 ? 0 : min(sq.n_kt, last_key / kTile + 1);
-  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarX), 1);
@@ -740,10 +877,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::kBarSFull + i), 1);
       mbar_init(bar(C::kBarB + i), 128);
+      mbar_init(bar(C::kBarItemFull + i), 1);
+      mbar_init(bar(C::kBarItemEmpty + i), kItemReaders);
     }
     mbar_init(bar(C::kBarDPFull), 1);
     mbar_init(bar(C::kBarDone), 1);
     mbar_init(bar(C::kBarDrain), 1);
+    mbar_init(bar(C::kBarXEmpty), 1);
+    mbar_init(bar(C::kBarAccEmpty), 256);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -756,11 +897,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, prm.wait_limit_ns};
-  const int qrow0 = sq.q0;  // first row of this sequence in the [rows, Hq, D] views
-  const int krow0 = sq.k0;  // and in the [rows, Hkv, D] views
+  const uint32_t full0 = bar(C::kBarItemFull), empty0 = bar(C::kBarItemEmpty);
 
   if (warp == kLoad) {
-    if (n_t > 0) {
     // ------------------------------------------------------------ loader (converged warp)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -769,44 +908,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
     }
     __syncwarp();
-    mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
-    for (int hf = 0; hf < C::kHalves; ++hf) {
-      tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, h, qrow0 + tile * kTile, bar(C::kBarX));
-      tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_do, hf * 64, h, qrow0 + tile * kTile, bar(C::kBarX));
-    }
-    int nk = 0, nv = 0;  // K and V tiles issued
-    for (int t = 0; t < n_t; ++t) {
-      const int row = krow0 + t * kTile;
-      const int sk = t % C::kKStages;
-      if (t >= C::kKStages &&
-          !warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((t / C::kKStages) & 1) ^ 1), wc))
-        break;
-      mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
-      for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, hk, row, bar(C::kBarKFull + sk));
-      nk = t + 1;
-      const int sv = t % C::kVStages;
-      if (t >= C::kVStages &&
-          !warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((t / C::kVStages) & 1) ^ 1), wc))
-        break;
-      mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
-      for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, hk, row, bar(C::kBarVFull + sv));
-      nv = t + 1;
+    int x = static_cast<int>(blockIdx.x);
+    int kc = 0, vc = 0, xi = 0;  // K and V tiles and (Q, dO) pairs loaded so far
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      ok = item_publish(item_slots, full0, empty0, i, x < prm.n_items ? x : -1, wc);
+      if (!ok || x >= prm.n_items) break;
+      const ItemQ it = item_q(prm, x);
+      if (it.n_t > 0) {
+        // Q, dO of this item once the previous item's last products have read theirs
+        if (xi > 0 && !(ok = warp_wait_bar(bar(C::kBarXEmpty), static_cast<uint32_t>((xi - 1) & 1), wc))) break;
+        const int qrow = it.sq.q0 + it.tile * kTile;
+        mbar_arrive_expect_tx_elect(bar(C::kBarX), 2 * C::kTileBytes);
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          tma_load_3d_elect(x_smem(0) + hf * C::kSlabBytes, &tm_q, hf * 64, it.h, qrow, bar(C::kBarX));
+          tma_load_3d_elect(x_smem(1) + hf * C::kSlabBytes, &tm_do, hf * 64, it.h, qrow, bar(C::kBarX));
+        }
+        ++xi;
+        for (int t = 0; t < it.n_t; ++t) {
+          const int row = it.sq.k0 + t * kTile;
+          const int sk = kc % C::kKStages;
+          if (kc >= C::kKStages &&
+              !(ok = warp_wait_bar(bar(C::kBarKEmpty + sk), static_cast<uint32_t>(((kc / C::kKStages) & 1) ^ 1), wc)))
+            break;
+          mbar_arrive_expect_tx_elect(bar(C::kBarKFull + sk), C::kTileBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_3d_elect(k_smem(sk) + hf * C::kSlabBytes, &tm_k, hf * 64, it.hk, row, bar(C::kBarKFull + sk));
+          ++kc;
+          const int sv = vc % C::kVStages;
+          if (vc >= C::kVStages &&
+              !(ok = warp_wait_bar(bar(C::kBarVEmpty + sv), static_cast<uint32_t>(((vc / C::kVStages) & 1) ^ 1), wc)))
+            break;
+          mbar_arrive_expect_tx_elect(bar(C::kBarVFull + sv), C::kTileBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_3d_elect(v_smem(sv) + hf * C::kSlabBytes, &tm_v, hf * 64, it.hk, row, bar(C::kBarVFull + sv));
+          ++vc;
+        }
+        if (!ok) break;
+      }
+      x = item_next(prm.sched, x, causal);
     }
     // let the copies this warp issued land before shared memory is released
-    drain_wait(bar(C::kBarX), 0);
-    for (int s = 0; s < C::kKStages && s < nk; ++s) {
-      const int tl = s + ((nk - 1 - s) / C::kKStages) * C::kKStages;
-      drain_wait(bar(C::kBarKFull + s), static_cast<uint32_t>((tl / C::kKStages) & 1));
+    if (xi > 0) drain_wait(bar(C::kBarX), static_cast<uint32_t>((xi - 1) & 1));
+    for (int s = 0; s < C::kKStages && s < kc; ++s) {
+      const int last = s + ((kc - 1 - s) / C::kKStages) * C::kKStages;
+      drain_wait(bar(C::kBarKFull + s), static_cast<uint32_t>((last / C::kKStages) & 1));
     }
-    for (int s = 0; s < C::kVStages && s < nv; ++s) {
-      const int tl = s + ((nv - 1 - s) / C::kVStages) * C::kVStages;
-      drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((tl / C::kVStages) & 1));
-    }
+    for (int s = 0; s < C::kVStages && s < vc; ++s) {
+      const int last = s + ((vc - 1 - s) / C::kVStages) * C::kVStages;
+      drain_wait(bar(C::kBarVFull + s), static_cast<uint32_t>((last / C::kVStages) & 1));
     }
   } else if (warp == kMma) {
-    if (n_t > 0) {
     // ------------------------------------------------------------ MMA issue (converged warp)
     constexpr uint32_t idesc_score = instr_desc_f16(kTile, kTile, FP16, false);
     constexpr uint32_t idesc_acc = instr_desc_f16(kTile, D, FP16, true);
@@ -824,128 +976,193 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ss_elect(tmem + col, a + off, bb + off, idesc_score, kk > 0 ? 1u : 0u);
       }
     };
-    auto issue_s = [&](int t) {  // S(t) = Q K_t^T into buffer t % 2
-      issue_score(q_desc, k_desc0 + static_cast<uint64_t>(t % C::kKStages) * kTileStep, C::kColS0 + 128 * (t & 1));
-      mma_commit_elect(bar(C::kBarSFull + (t & 1)));
+    int kc = 0, vc = 0, tc = 0, xi = 0;  // K, V tiles, score tiles and items with work so far
+    // S(t) = Q K_t^T into buffer (tc + t) % 2; dP(t) = dO V_t^T
+    auto issue_s = [&](int t) {
+      const int b = (tc + t) & 1;
+      issue_score(q_desc, k_desc0 + static_cast<uint64_t>((kc + t) % C::kKStages) * kTileStep, C::kColS0 + 128 * b);
+      mma_commit_elect(bar(C::kBarSFull + b));
     };
-    auto issue_dp = [&](int t) {  // dP(t) = dO V_t^T
-      issue_score(do_desc, v_desc0 + static_cast<uint64_t>(t % C::kVStages) * kTileStep, C::kColDP);
+    auto issue_dp = [&](int t) {
+      issue_score(do_desc, v_desc0 + static_cast<uint64_t>((vc + t) % C::kVStages) * kTileStep, C::kColDP);
       mma_commit_elect(bar(C::kBarDPFull));
     };
-    bool ok = warp_wait_bar(bar(C::kBarX), 0, wc) && warp_wait_bar(bar(C::kBarKFull), 0, wc);
-    if (ok) {
-      tc_fence_after();
-      issue_s(0);
-      ok = warp_wait_bar(bar(C::kBarVFull), 0, wc);
-    }
-    if (ok) {
-      tc_fence_after();
-      issue_dp(0);
-      if (n_t > 1) {
-        ok = warp_wait_bar(bar(C::kBarKFull + 1), 0, wc);
-        if (ok) {
-          tc_fence_after();
-          issue_s(1);
-        }
+    auto wait_k = [&](int t) {
+      return warp_wait_bar(bar(C::kBarKFull + (kc + t) % C::kKStages),
+                           static_cast<uint32_t>(((kc + t) / C::kKStages) & 1), wc);
+    };
+    auto wait_v = [&](int t) {
+      return warp_wait_bar(bar(C::kBarVFull + (vc + t) % C::kVStages),
+                           static_cast<uint32_t>(((vc + t) / C::kVStages) & 1), wc);
+    };
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int x = item_take(item_slots, full0, empty0, i, wc);
+      if (x < 0) {
+        ok = x == -1;
+        break;
       }
-    }
-    for (int t = 0; ok && t < n_t; ++t) {
-      const uint32_t ph = static_cast<uint32_t>(t & 1);
-      // both warpgroups have read dP(t) and written dS(t) into S buffer t % 2
-      ok = warp_wait_bar(bar(C::kBarB), ph, wc) && warp_wait_bar(bar(C::kBarB + 1), ph, wc);
+      const ItemQ it = item_q(prm, x);
+      const int n = it.n_t;
+      if (n == 0) continue;
+      ok = warp_wait_bar(bar(C::kBarX), static_cast<uint32_t>(xi & 1), wc) && wait_k(0);
       if (!ok) break;
       tc_fence_after();
-      mma_commit_elect(bar(C::kBarVEmpty + t % C::kVStages));  // V_t: its reader dP(t) is done
-      if (t + 1 < n_t) {
-        ok = warp_wait_bar(bar(C::kBarVFull + (t + 1) % C::kVStages), static_cast<uint32_t>(((t + 1) / C::kVStages) & 1),
-                           wc);
+      issue_s(0);
+      if (!(ok = wait_v(0))) break;
+      tc_fence_after();
+      issue_dp(0);
+      if (n == 1) mma_commit_elect(bar(C::kBarXEmpty));  // Q, dO of this item: last readers issued
+      if (n > 1) {
+        if (!(ok = wait_k(1))) break;
+        tc_fence_after();
+        issue_s(1);
+      }
+      for (int t = 0; ok && t < n; ++t) {
+        const uint32_t ph = static_cast<uint32_t>((tc + t) & 1);
+        // both warpgroups have read dP(t) and written dS(t) into its S buffer
+        ok = warp_wait_bar(bar(C::kBarB), ph, wc) && warp_wait_bar(bar(C::kBarB + 1), ph, wc);
         if (!ok) break;
         tc_fence_after();
-        issue_dp(t + 1);
-      }
-      // dQ += dS(t) K_t: A = dS pairs in S buffer t % 2 (warpgroup h: columns 64h ..), B = K_t MN-major
-      const uint64_t kb = k_mn0 + static_cast<uint64_t>(t % C::kKStages) * kTileStep;
-      const uint32_t a0 = C::kColS0 + 128 * (t & 1);
+        mma_commit_elect(bar(C::kBarVEmpty + (vc + t) % C::kVStages));  // V_t: its reader dP(t) is done
+        if (t + 1 < n) {
+          if (!(ok = wait_v(t + 1))) break;
+          tc_fence_after();
+          issue_dp(t + 1);
+          if (t + 1 == n - 1) mma_commit_elect(bar(C::kBarXEmpty));
+        }
+        // the item's first dQ product overwrites the accumulator: the previous
+        // item's dQ must have been read out
+        if (t == 0 && xi > 0) {
+          if (!(ok = warp_wait_bar(bar(C::kBarAccEmpty), static_cast<uint32_t>((xi - 1) & 1), wc))) break;
+          tc_fence_after();
+        }
+        // dQ += dS(t) K_t: A = dS pairs in its S buffer (warpgroup h: columns 64h ..), B = K_t MN-major
+        const uint64_t kb = k_mn0 + static_cast<uint64_t>((kc + t) % C::kKStages) * kTileStep;
+        const uint32_t a0 = C::kColS0 + 128 * ((tc + t) & 1);
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        mma_ts_elect(tmem + C::kColAcc, tmem + a0 + 64 * (kk / 4) + 8 * (kk % 4), kb + static_cast<uint64_t>(kk * (2048 >> 4)),
-                     idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          mma_ts_elect(tmem + C::kColAcc, tmem + a0 + 64 * (kk / 4) + 8 * (kk % 4),
+                       kb + static_cast<uint64_t>(kk * (2048 >> 4)), idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit_elect(bar(C::kBarKEmpty + (kc + t) % C::kKStages));  // K_t: last reader issued
+        if (t + 2 < n) {
+          if (!(ok = wait_k(t + 2))) break;
+          tc_fence_after();
+          issue_s(t + 2);  // into the buffer of S(t), after dQ(t) has read dS(t) from it (in order)
+        }
+        if (t == n - 1) mma_commit_elect(bar(C::kBarDone));
       }
-      mma_commit_elect(bar(C::kBarKEmpty + t % C::kKStages));  // K_t: last reader issued
-      if (t + 2 < n_t) {
-        ok = warp_wait_bar(bar(C::kBarKFull + (t + 2) % C::kKStages), static_cast<uint32_t>(((t + 2) / C::kKStages) & 1),
-                           wc);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(t + 2);  // into buffer t % 2, after dQ(t) has read dS(t) from it (in order)
-      }
-      if (t == n_t - 1) mma_commit_elect(bar(C::kBarDone));
+      kc += n;
+      vc += n;
+      tc += n;
+      ++xi;
     }
     if (!ok) {
       mma_commit_elect(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0);
-    }
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups (TMEM lane = row)
     const int wg = warp / 4;                  // column half of every score tile
     const int qd = warp % 4;                  // TMEM lane quadrant
     const int row = qd * 32 + lane;
-    const int r_abs = tile * kTile + row;     // this thread's query
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const float c = prm.scale_log2;
-    const float nl_row = prm.ws_l[static_cast<int64_t>(bh) * prm.Npad + r_abs];
-    const float nd_row = prm.ws_d[static_cast<int64_t>(bh) * prm.Npad + r_abs];
+    int tc = 0, xi = 0;
     bool ok = true;
-    for (int t = 0; t < n_t; ++t) {
-      const int first_col = t * kTile + 64 * wg;  // first key of this warpgroup's half
-      const uint32_t t_s = tmem + lane_base + C::kColS0 + 128 * (t & 1) + 64 * wg;
-      // masked: the causal boundary cuts the tile (its last key is not seen by
-      // the tile's first query), or the keys run out
-      const bool masked = (causal && t * kTile + kTile - 1 > tile * kTile + sq.delta) || (t + 1) * kTile > sq.nk;
-      ok = warp_wait_bar(bar(C::kBarSFull + (t & 1)), static_cast<uint32_t>((t >> 1) & 1), wc);
-      if (!ok) break;
-      tc_fence_after();
-      float p[64];
-      if (masked) {
-        phase_a<FP16, false, true, false>(t_s, c, nl_row, nullptr, first_col, r_abs, sq.nk, causal, sq.delta, p);
-      } else {
-        phase_a<FP16, false, false, false>(t_s, c, nl_row, nullptr, first_col, r_abs, sq.nk, causal, sq.delta, p);
-      }
-      ok = warp_wait_bar(bar(C::kBarDPFull), static_cast<uint32_t>(t & 1), wc);
-      if (!ok) break;
-      tc_fence_after();
-      // dS pairs over the first 32 columns of this half of S(t) (read above)
-      phase_b<FP16, false>(tmem + lane_base + C::kColDP + 64 * wg, t_s, nd_row, nullptr, p);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarB + wg));
-    }
-    if (ok && n_t > 0) ok = warp_wait_bar(bar(C::kBarDone), 0, wc);
-    if (ok) {
-      tc_fence_after();
-      // warpgroup h writes dQ columns h D/2 .. (scaled); a tile whose queries
-      // see no key at all gets 0
-      const bool row_valid =
-          r_abs < sq.nq && index_ok(static_cast<int64_t>(sq.q0) + r_abs < prm.total_q && h < prm.Hq);
-      uint16_t* dst_row = prm.out0 + ((static_cast<int64_t>(sq.q0) + r_abs) * prm.Hq + h) * D + wg * (D / 2);
-      const uint32_t acc = tmem + lane_base + C::kColAcc + wg * (D / 2);
-#pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        uint32_t a[32];
-        tmem_ld32(acc + q * 32, a);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pk[k] = n_t > 0 ? pack2<FP16>(__uint_as_float(a[2 * k]) * prm.scale, __uint_as_float(a[2 * k + 1]) * prm.scale)
-                          : 0u;
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+    // this thread's -LSE log2(e) and -D for item x (loaded ahead of use)
+    auto row_values = [&](int x, float& nl, float& nd) {
+      nl = 0.f;
+      nd = 0.f;
+      if (x < 0) return;
+      const ItemQ it = item_q(prm, x);
+      if (it.skip) return;
+      const int64_t at = static_cast<int64_t>(it.bh) * prm.Npad + it.tile * kTile + row;
+      nl = prm.ws_l[at];
+      nd = prm.ws_d[at];
+    };
+    int x = item_take(item_slots, full0, empty0, 0, wc);
+    float nl_row, nd_row;
+    row_values(x, nl_row, nd_row);
+    for (int i = 0; x >= 0; ++i) {
+      const ItemQ it = item_q(prm, x);
+      const int r_abs = it.tile * kTile + row;  // this thread's query
+      if (!it.skip) {
+        for (int t = 0; t < it.n_t; ++t) {
+          const int T = tc + t;
+          const int first_col = t * kTile + 64 * wg;  // first key of this warpgroup's half
+          const uint32_t t_s = tmem + lane_base + C::kColS0 + 128 * (T & 1) + 64 * wg;
+          // masked: the causal boundary cuts the tile (its last key is not seen by
+          // the tile's first query), or the keys run out
+          const bool masked =
+              (causal && t * kTile + kTile - 1 > it.tile * kTile + it.sq.delta) || (t + 1) * kTile > it.sq.nk;
+          ok = warp_wait_bar(bar(C::kBarSFull + (T & 1)), static_cast<uint32_t>((T >> 1) & 1), wc);
+          if (!ok) break;
+          tc_fence_after();
+          float p[64];
+          if (masked) {
+            phase_a<FP16, false, true, false>(t_s, c, nl_row, nullptr, first_col, r_abs, it.sq.nk, causal,
+                                              it.sq.delta, p);
+          } else {
+            phase_a<FP16, false, false, false>(t_s, c, nl_row, nullptr, first_col, r_abs, it.sq.nk, causal,
+                                               it.sq.delta, p);
+          }
+          ok = warp_wait_bar(bar(C::kBarDPFull), static_cast<uint32_t>(T & 1), wc);
+          if (!ok) break;
+          tc_fence_after();
+          // dS pairs over the first 32 columns of this half of S(t) (read above)
+          phase_b<FP16, false>(tmem + lane_base + C::kColDP + 64 * wg, t_s, nd_row, nullptr, p);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::kBarB + wg));
         }
+        if (!ok) break;
+      } else if (!it.sq.ok && threadIdx.x == 0) {
+        atomicOr(&g_status_word, 2u);  // inconsistent packed offsets
       }
+      // the next item (published by now: this item's loads have all been
+      // issued); its rows' values load while this item's dQ is written out
+      const int nx = item_take(item_slots, full0, empty0, i + 1, wc);
+      float nl_next, nd_next;
+      row_values(nx, nl_next, nd_next);
+      if (!it.skip) {
+        if (it.n_t > 0 && !(ok = warp_wait_bar(bar(C::kBarDone), static_cast<uint32_t>(xi & 1), wc))) break;
+        // warpgroup h writes dQ columns h D/2 .. (scaled); a tile whose queries
+        // see no key at all gets 0. After the last read of the accumulator it
+        // goes back to the MMA warp.
+        const bool row_valid =
+            r_abs < it.sq.nq && index_ok(static_cast<int64_t>(it.sq.q0) + r_abs < prm.total_q && it.h < prm.Hq);
+        uint16_t* dst_row =
+            prm.out0 + ((static_cast<int64_t>(it.sq.q0) + r_abs) * prm.Hq + it.h) * D + wg * (D / 2);
+        const uint32_t acc = tmem + lane_base + C::kColAcc + wg * (D / 2);
+        if (it.n_t > 0) tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < D / 64; ++q) {
+          uint32_t pk[16];
+          if (it.n_t > 0) {
+            uint32_t a[32];
+            tmem_ld32(acc + q * 32, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              pk[k] = pack2<FP16>(__uint_as_float(a[2 * k]) * prm.scale, __uint_as_float(a[2 * k + 1]) * prm.scale);
+            if (q == D / 64 - 1) {
+              tc_fence_before();
+              mbar_arrive(bar(C::kBarAccEmpty));
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+          }
+          if (row_valid) store_row64(dst_row + q * 32, pk, prm.wide_stores != 0);
+        }
+        tc += it.n_t;
+        if (it.n_t > 0) ++xi;
+      }
+      x = nx;
+      nl_row = nl_next;
+      nd_row = nd_next;
     }
   }
 

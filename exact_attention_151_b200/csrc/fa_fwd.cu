@@ -336,9 +336,11 @@ Shape dense_shape(int64_t B, int64_t Nq, int64_t Nk, int64_t Hq, int64_t Hkv, in
 
 // Workspace of the backward: D_i = dO_i . O_i, then LSE_i log2(e), each fp32
 // [B*Hq, Npad] with Npad = Nq rounded up to whole 128-row tiles, 256-byte aligned.
+// -D and -LSE log2(e) per padded row, then the two gradient kernels' work-item counters
 size_t bwd_ws_bytes(int64_t B, int64_t Nq, int64_t Hq) {
+  if (B <= 0 || Hq <= 0) return 0;  // nothing to do
   const int64_t npad = (Nq + kTile - 1) / kTile * kTile;
-  return 2 * align256(static_cast<size_t>(B * Hq * npad) * 4);
+  return 2 * align256(static_cast<size_t>(B * Hq * npad) * 4) + 256;
 }
 
 template <int D, bool FP16, bool KV_SIDE>
@@ -394,8 +396,8 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
   const int64_t npad = n_qt * kTile;
   const int64_t BHq = B * Hq;
   float* ws_d = static_cast<float*>(workspace);
-  float* ws_l = ws_d ? reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BHq * npad) * 4))
-                     : nullptr;
+  float* ws_l = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(BHq * npad) * 4));
+  int* sched = reinterpret_cast<int*>(static_cast<char*>(workspace) + 2 * align256(static_cast<size_t>(BHq * npad) * 4));
   constexpr int64_t kPrepRows = 256 / (D / 8);  // rows per preprocess block
   const int64_t real_blocks = (tq_rows * Hq + kPrepRows - 1) / kPrepRows;
   const int64_t pad_blocks = sh.cu_q ? (BHq * npad + 255) / 256 : (BHq * (npad - Nq) + 255) / 256;
@@ -405,15 +407,22 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
       bwd::fa_bwd_prep_varlen_kernel<D, FP16><<<grid, 256, 0, stream>>>(
           static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, sh.cu_q,
           static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(tq_rows), static_cast<int>(npad),
-          static_cast<unsigned>(real_blocks));
+          static_cast<unsigned>(real_blocks), sched);
     } else {
       bwd::fa_bwd_prep_kernel<D, FP16><<<grid, 256, 0, stream>>>(
           static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(B),
-          static_cast<int>(Nq), static_cast<int>(Hq), static_cast<int>(npad), static_cast<unsigned>(real_blocks));
+          static_cast<int>(Nq), static_cast<int>(Hq), static_cast<int>(npad), static_cast<unsigned>(real_blocks),
+          sched);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       set_error("backward preprocess launch", e);
+      return FA_ERR_CUDA;
+    }
+  } else {
+    const cudaError_t e = cudaMemsetAsync(sched, 0, 2 * sizeof(int), stream);  // no rows to preprocess
+    if (e != cudaSuccess) {
+      set_error("cudaMemsetAsync(backward work-item counters)", e);
       return FA_ERR_CUDA;
     }
   }
@@ -450,24 +459,35 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
   prm.scale = scale;
   prm.causal = causal ? 1 : 0;
   prm.wait_limit_ns = kDefaultWaitLimitNs;
-  // query side: one CTA per (query tile, b, query head)
+  // rows are D * 2 bytes apart (a multiple of 128): 32-byte stores if the bases allow
+  auto aligned32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };
+  // persistent grids: one CTA per SM, at most one per work item
+  const int64_t sms = device_sm_count(dev);
+  // query side: work items (query tile, b, query head)
   prm.out0 = static_cast<uint16_t*>(dq);
   prm.out1 = nullptr;
   prm.BH = static_cast<int>(BHq);
   prm.n_tiles = static_cast<int>(n_qt);
-  fa_status st = bwd_launch<D, FP16, false>(dev, tq, tdo, tk, tv, prm, n_qt * BHq, stream);
+  prm.n_items = static_cast<int>(n_qt * BHq);
+  prm.sched = sched;
+  prm.wide_stores = aligned32(dq) ? 1 : 0;
+  fa_status st = bwd_launch<D, FP16, false>(dev, tq, tdo, tk, tv, prm, std::min<int64_t>(prm.n_items, sms), stream);
   if (st != FA_OK) return st;
-  // key side: one CTA per (key tile, b, K/V head)
+  // key side: work items (key tile, b, K/V head)
   prm.out0 = static_cast<uint16_t*>(dk);
   prm.out1 = static_cast<uint16_t*>(dv);
   prm.BH = static_cast<int>(B * Hkv);
   prm.n_tiles = static_cast<int>(n_kt);
-  st = bwd_launch<D, FP16, true>(dev, tk, tv, tq, tdo, prm, n_kt * B * Hkv, stream);
+  prm.n_items = static_cast<int>(n_kt * B * Hkv);
+  prm.sched = sched + 1;
+  prm.wide_stores = aligned32(dk) && aligned32(dv) ? 1 : 0;
+  st = bwd_launch<D, FP16, true>(dev, tk, tv, tq, tdo, prm, std::min<int64_t>(prm.n_items, sms), stream);
   if (st != FA_OK) return st;
   if (debug_enabled())
-    std::fprintf(stderr, "[fa] bwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d grid=%lld+%lld\n", D,
-                 FP16 ? "fp16" : "bf16", (long long)B, (long long)Nq, (long long)Nk, (long long)Hq, (long long)Hkv,
-                 sh.cu_q ? "packed" : "dense", causal, (long long)(n_qt * BHq), (long long)(n_kt * B * Hkv));
+    std::fprintf(stderr, "[fa] bwd D=%d %s B=%lld Nq=%lld Nk=%lld Hq=%lld Hkv=%lld %s causal=%d items=%lld+%lld on %lld SMs\n",
+                 D, FP16 ? "fp16" : "bf16", (long long)B, (long long)Nq, (long long)Nk, (long long)Hq, (long long)Hkv,
+                 sh.cu_q ? "packed" : "dense", causal, (long long)(n_qt * BHq), (long long)(n_kt * B * Hkv),
+                 (long long)sms);
   return FA_OK;
 }
 

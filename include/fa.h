@@ -227,8 +227,10 @@ fa_status fa_status_sync(fa_stream_t stream);
 
 /*
  * fa_bwd_workspace_size - bytes of device workspace fa_bwd needs for these
- * sizes: two fp32 arrays [B*H, ceil(N/128)*128], each rounded up to 256 bytes.
- * For fa_bwd_gqa pass the query side's sizes (B, Nq, Hq).
+ * sizes: two fp32 arrays [B*H, ceil(N/128)*128], each rounded up to 256 bytes,
+ * then 256 bytes for the gradient kernels' work-item counters (0 in all when
+ * B or H is 0: there is nothing to do). For fa_bwd_gqa pass the query side's
+ * sizes (B, Nq, Hq).
  * Returns FA_ERR_INVALID_ARG for a NULL output or a negative size.
  */
 fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspace_bytes);
@@ -257,10 +259,12 @@ fa_status fa_bwd_workspace_size(int64_t B, int64_t N, int64_t H, size_t* workspa
  *   workspace        : device, at least fa_bwd_workspace_size(B, N, H) bytes,
  *                      256-byte aligned; owned by the caller, scratch for the
  *                      duration of the call (stream-ordered)
- * Three kernels run in stream order: D and LSE log2(e) into the workspace,
- * then dQ (one CTA per 128-query tile), then dK and dV (one CTA per 128-key
- * tile). fp32 accumulation in Tensor Memory; P and dS enter the tensor cores
- * rounded to `dtype`.
+ * Three kernels run in stream order: D and LSE log2(e) into the workspace
+ * (which also resets the work-item counters), then dQ (work items of 128
+ * queries), then dK and dV (work items of 128 keys); the last two are
+ * persistent, one CTA per SM taking items from its counter, and an item's
+ * result does not depend on which CTA computed it. fp32 accumulation in
+ * Tensor Memory; P and dS enter the tensor cores rounded to `dtype`.
  * Errors: as fa_fwd; additionally FA_ERR_INVALID_ARG for a NULL or too small
  * workspace and FA_ERR_MISALIGNED for a workspace not 256-byte aligned.
  * B, N or H == 0 returns FA_OK without launching.

@@ -108,9 +108,11 @@ def test_backward_validates_before_any_device_call():
 
 
 def test_backward_workspace_size():
-    # two fp32 arrays [B*H, N rounded up to 128], each rounded up to 256 bytes
-    assert fa.bwd_workspace_size(2, 300, 3) == 2 * (2 * 3 * 384 * 4)
-    assert fa.bwd_workspace_size(1, 1, 1) == 2 * 512
+    # two fp32 arrays [B*H, N rounded up to 128], each rounded up to 256 bytes,
+    # then 256 bytes of work-item counters
+    assert fa.bwd_workspace_size(2, 300, 3) == 2 * (2 * 3 * 384 * 4) + 256
+    assert fa.bwd_workspace_size(1, 1, 1) == 2 * 512 + 256
+    assert fa.bwd_workspace_size(2, 0, 3) == 256  # no queries: the key side still runs (zero dK, dV)
     assert fa.bwd_workspace_size(0, 5, 5) == 0
     lib = fa.load_library()
     import ctypes

@@ -189,3 +189,27 @@ def test_packed_inconsistent_offsets_are_reported():
     fa.bwd_varlen(q, q, q, o, lse, q, cu_q, cu_k, 60, 40, causal=False)
     assert fa.status_sync() == fa.FA_ERR_INVALID_ARG
     assert fa.status_sync() == fa.FA_OK
+
+
+def test_gradients_at_16_byte_offsets_match_aligned_bitwise():
+    """Gradient buffers that are only 16-byte aligned take the 16-byte store
+    path of the epilogues (32-byte aligned ones the 32-byte path); both write
+    the same bits."""
+    B, N, Hq, Hkv, D = 2, 300, 4, 2, 128
+    g = torch.Generator().manual_seed(41)
+    q, do = (torch.randn(B, N, Hq, D, generator=g).to(torch.bfloat16).to(DEV) for _ in range(2))
+    k, v = (torch.randn(B, N, Hkv, D, generator=g).to(torch.bfloat16).to(DEV) for _ in range(2))
+    o, lse = fa.fwd(q, k, v, causal=True)
+    a = fa.bwd(q, k, v, o, lse, do, causal=True)
+
+    def offset_like(t):  # a view 16 bytes past a 256-byte aligned allocation
+        buf = torch.full((t.numel() + 8,), float("nan"), dtype=t.dtype, device=DEV)
+        view = buf[8:].view(t.shape)
+        assert view.data_ptr() % 32 == 16
+        return view
+
+    dq, dk, dv = offset_like(q), offset_like(k), offset_like(k)
+    fa.bwd(q, k, v, o, lse, do, causal=True, dq=dq, dk=dk, dv=dv)
+    assert fa.status_sync() == fa.FA_OK
+    for x, y in zip(a, (dq, dk, dv)):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))

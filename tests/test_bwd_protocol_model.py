@@ -1,27 +1,36 @@
 """Models of the backward kernels' mbarrier protocols, run under random schedules.
 
-They mirror the hand-offs of `fa_bwd_dkdv_kernel` and `fa_bwd_dq_kernel`
-(exact_attention_151_b200/csrc/fa_bwd_kernel.cuh), not their arithmetic. Each has
-a loader warp, an MMA warp issuing in the kernel's order, and two compute
-warpgroups (one per 64-column half of every score tile) of four warps; the
-kernels' 128-thread arrivals are four warp arrivals here.
+They mirror the hand-offs of the persistent `fa_bwd_dkdv_kernel` and
+`fa_bwd_dq_kernel` (exact_attention_151_b200/csrc/fa_bwd_kernel.cuh), not their
+arithmetic. A CTA has a loader warp, an MMA warp issuing in the kernel's order,
+and two compute warpgroups (one per 64-column half of every score tile) of four
+warps; the kernels' 128-thread arrivals are four warp arrivals here (256-thread
+ones eight). The CTA works through a sequence of items (the scheduler's choice
+does not matter to the protocol), each with its own number of streamed tiles,
+zero included (an item whose gradients are zero: no loads, no products).
 
-dK/dV (one key tile, n query tiles t): the loader brings K, V once and, per t,
-Q_t, dO_t and the -LSE / -D rows into stage t % 2. The MMA warp issues S^T(0) and
-dP^T(0), then per t: dV += P^T dO per half (after that half's phase A), S^T(t+1)
-over the P^T columns, dK += dS^T Q per half (after phase B), the stage release,
-and dP^T(t+1) over the dS^T columns (or the final commit). A warpgroup waits for
-the stage and S^T(t), runs phase A (P^T in place), then waits for dP^T(t) and
-runs phase B (dS^T in place, reading the stage's -D row).
+Items: the loader publishes each into a two-slot ring (ItemFull / ItemEmpty,
+read by the MMA warp and the eight compute warps) and ends with -1. Ring
+stages, score buffers and the phases of every barrier are counted across
+items. The fixed operands of an item (dK/dV: K and V; dQ: Q and dO) are
+reloaded once the previous item's last products reading them have completed
+(XEmpty); the accumulators are reused once the compute warps have read the
+previous item's out (AccEmpty).
 
-dQ (one query tile, n key tiles t): K_t into a 3-stage ring, V_t into a 2-stage
-ring. The MMA warp issues S(0) (buffer 0), dP(0), S(1) (buffer 1), then per t:
-after both warpgroups' phase B, releases V_t, issues dP(t+1), dQ += dS(t) K_t
-(A = dS in S buffer t % 2), releases K_t, and issues S(t+2) into buffer t % 2.
+dK/dV: per item, the MMA warp issues S^T(0) and dP^T(0), then per tile t:
+dV += P^T dO per half (after that half's phase A), S^T(t+1) over the P^T
+columns, dK += dS^T Q per half (after phase B), the stage release, and dP^T(t+1)
+over the dS^T columns (or the item's final commit).
+
+dQ: K_t into a 3-stage ring, V_t into a 2-stage ring. Per item the MMA warp
+issues S(0), dP(0), S(1), then per tile t: after both warpgroups' phase B,
+releases V_t, issues dP(t+1), dQ += dS(t) K_t, releases K_t, and issues S(t+2)
+into the buffer of S(t).
 
 Checked: no waiter more than one phase behind; nothing in TMEM or shared memory
-overwritten before its last reader has finished; readers find what they expect;
-no deadlock. Planted bugs must fail, or the models would prove nothing.
+(stages, fixed operands, item slots, accumulators) overwritten before its last
+reader has finished; readers find what they expect; no deadlock. Planted bugs
+must fail, or the models would prove nothing.
 """
 
 import random
@@ -32,133 +41,231 @@ from tests.protocol_sim import Model, ProtocolError
 
 STAGES_DKDV = 2
 K_STAGES_DQ, V_STAGES_DQ = 3, 2
+ITEM_READERS = 9  # the MMA warp and the eight compute warps
 
 
-def simulate_dkdv(n_t, seed, plant=None):
+class ItemRing:
+    """The two-slot work-item ring: the loader publishes, nine warps read."""
+
+    def __init__(self, m, seq, plant):
+        self.m, self.seq, self.plant = m, seq, plant
+        self.slots = [None, None]
+        self.unread = [0, 0]
+        for s in range(2):
+            m.bar(f"IF{s}")
+            m.bar(f"IE{s}", ITEM_READERS)
+
+    def publish(self, i):
+        slot = i & 1
+        if i >= 2 and self.plant != "slot_early":
+            yield from self.m.wait(f"IE{slot}", (i >> 1) - 1)
+        if self.unread[slot]:
+            raise ProtocolError(f"item slot {slot} overwritten before every warp read item {i - 2}")
+        self.slots[slot] = (i, self.seq[i])
+        self.unread[slot] = ITEM_READERS
+        self.m.bars[f"IF{slot}"].arrive()
+
+    def take(self, i):
+        slot = i & 1
+        yield from self.m.wait(f"IF{slot}", i >> 1)
+        idx, n = self.slots[slot]
+        if idx != i:
+            raise ProtocolError(f"a warp expecting item {i} read item {idx}")
+        self.unread[slot] -= 1
+        self.m.bars[f"IE{slot}"].arrive()
+        return n
+
+
+def simulate_dkdv(items, seed, plant=None):
+    """items: streamed-tile counts of the CTA's items, in order (0: no work)."""
     m = Model(seed)
-    m.bar("X")
+    seq = list(items) + [-1]
+    ring = ItemRing(m, seq, plant)
+    for name in ("X", "XE", "SF", "DPF", "Done", "Drain"):
+        m.bar(name)
+    m.bar("AccE", 8)
     for s in range(STAGES_DKDV):
         m.bar(f"YF{s}")
         m.bar(f"YE{s}")
-    for name in ("SF", "DPF", "Done"):
-        m.bar(name)
     for h in range(2):
         m.bar(f"A{h}", 4)
         m.bar(f"B{h}", 4)
-    stage = [None] * STAGES_DKDV
+    stage = [None] * STAGES_DKDV   # global streamed tile held
     landed = [False] * STAGES_DKDV
-    readers = {}  # stage item t -> MMA ids reading it
-    ws_users = {}  # stage item t -> warps still reading its -LSE / -D rows
-    s_cols, dp_cols = {"t": None}, {"t": None}
+    xbuf = {"item": None, "landed": False}
+    readers = {}     # ("Y", g) / ("X", xi) -> MMA ids reading it
+    ws_users = {}    # g -> warps still reading the stage's -LSE / -D rows
+    s_cols, dp_cols = {"T": None}, {"T": None}
     wrote_p, wrote_ds = {}, {}
+    acc = {"item": None, "last": -1, "read": {}}  # item accumulating; last MMA id into it; warps that read item xi
     state = {}
 
+    def busy(key):
+        return any(i >= m.done for i in readers.get(key, []))
+
     def loader():
-        m.later(lambda: m.bars["X"].arrive())
-        for t in range(n_t):
-            s = t % STAGES_DKDV
-            if t >= STAGES_DKDV:
-                yield from m.wait(f"YE{s}", t // STAGES_DKDV - 1)
-                if any(i >= m.done for i in readers.get(t - STAGES_DKDV, [])):
-                    raise ProtocolError(f"stage {s} reloaded while an MMA reads tile {t - STAGES_DKDV}")
-                if ws_users.get(t - STAGES_DKDV):
-                    raise ProtocolError(f"stage {s} reloaded while a warp reads tile {t - STAGES_DKDV}'s rows")
-            stage[s], landed[s] = t, False
-
-            def land(s=s):
-                landed[s] = True
-                m.bars[f"YF{s}"].arrive()
-            m.later(land)
+        yc = xi = 0
+        for i, n in enumerate(seq):
+            yield from ring.publish(i)
             yield
+            if n < 0:
+                return
+            if n == 0:
+                continue
+            if xi > 0 and plant != "x_early":
+                yield from m.wait("XE", xi - 1)
+            if busy(("X", xi - 1)):
+                raise ProtocolError(f"K, V of item {xi} loaded while item {xi - 1}'s products read theirs")
+            xbuf["item"], xbuf["landed"] = xi, False
 
-    def score(cols, t, what):
-        s = t % STAGES_DKDV
-        if stage[s] != t or not landed[s]:
-            raise ProtocolError(f"{what}({t}) reads a stage without tile {t}")
-        if cols["t"] is not None:
-            prev = cols["t"]
+            def land_x(xi=xi):
+                xbuf["landed"] = True
+                m.bars["X"].arrive()
+            m.later(land_x)
+            xi += 1
+            for _ in range(n):
+                s = yc % STAGES_DKDV
+                if yc >= STAGES_DKDV:
+                    yield from m.wait(f"YE{s}", yc // STAGES_DKDV - 1)
+                    if busy(("Y", yc - STAGES_DKDV)):
+                        raise ProtocolError(f"stage {s} reloaded while an MMA reads tile {yc - STAGES_DKDV}")
+                    if ws_users.get(yc - STAGES_DKDV):
+                        raise ProtocolError(f"stage {s} reloaded while a warp reads tile {yc - STAGES_DKDV}'s rows")
+                stage[s], landed[s] = yc, False
+
+                def land(s=s):
+                    landed[s] = True
+                    m.bars[f"YF{s}"].arrive()
+                m.later(land)
+                yc += 1
+                yield
+
+    def score(cols, g, T, xi, what):
+        s = g % STAGES_DKDV
+        if stage[s] != g or not landed[s]:
+            raise ProtocolError(f"{what}({T}) reads a stage without tile {g}")
+        if xbuf["item"] != xi or not xbuf["landed"]:
+            raise ProtocolError(f"{what}({T}) reads K, V without item {xi}'s")
+        if cols["T"] is not None:
+            prev = cols["T"]
             if not state.get((what, prev, "read")):
-                raise ProtocolError(f"{what}({t}) overwrites {what}({prev}) before both warpgroups read it")
-            # P^T (dS^T) of tile prev sits in these columns until the dV (dK) MMAs
-            # that read it are issued; one thread's MMAs run in order
+                raise ProtocolError(f"{what}({T}) overwrites {what}({prev}) before both warpgroups read it")
+            # P^T (dS^T) of tile prev sits in these columns until the dV (dK)
+            # MMAs that read it are issued; one thread's MMAs run in order
             reader = "dV" if what == "S" else "dK"
             if not (state.get((reader, prev, 0)) and state.get((reader, prev, 1))):
-                raise ProtocolError(f"{what}({t}) overwrites the operand of {reader}({prev}) before it is issued")
+                raise ProtocolError(f"{what}({T}) overwrites the operand of {reader}({prev}) before it is issued")
         ids = [m.mma() for _ in range(8)]
-        readers.setdefault(t, []).extend(ids)
-        cols["t"] = t
+        readers.setdefault(("Y", g), []).extend(ids)
+        readers.setdefault(("X", xi), []).extend(ids)
+        cols["T"] = T
 
-    def acc(t, h, kind):
-        if not (wrote_p if kind == "dV" else wrote_ds).get((t, h)):
-            raise ProtocolError(f"{kind}({t}) half {h} before its operand was written")
+    def accumulate(g, T, h, kind, xi, first):
+        if not (wrote_p if kind == "dV" else wrote_ds).get((T, h)):
+            raise ProtocolError(f"{kind}({T}) half {h} before its operand was written")
+        if first and xi > 0 and acc["read"].get(xi - 1, 0) < 8:
+            raise ProtocolError(f"item {xi}'s first {kind} overwrites item {xi - 1}'s accumulators before they are read")
         ids = [m.mma() for _ in range(4)]
-        readers.setdefault(t, []).extend(ids)
-        state[(kind, t, h)] = True
+        readers.setdefault(("Y", g), []).extend(ids)
+        acc["item"], acc["last"] = xi, ids[-1]
+        state[(kind, T, h)] = True
 
     def mma_warp():
-        yield from m.wait("X", 0)
-        yield from m.wait("YF0", 0)
-        score(s_cols, 0, "S")
-        m.commit("SF")
-        score(dp_cols, 0, "dP")
-        m.commit("DPF")
-        yield
-        for t in range(n_t):
-            s = t % STAGES_DKDV
-            more = t + 1 < n_t
-            if more and plant == "s_over_p":
-                yield from m.wait(f"YF{(t + 1) % STAGES_DKDV}", (t + 1) // STAGES_DKDV)
-                score(s_cols, t + 1, "S")
-                m.commit("SF")
-            for h in range(2):
-                yield from m.wait(f"A{h}", t)
-                acc(t, h, "dV")
-                yield
-            if more and plant != "s_over_p":
-                yield from m.wait(f"YF{(t + 1) % STAGES_DKDV}", (t + 1) // STAGES_DKDV)
-                score(s_cols, t + 1, "S")
-                m.commit("SF")
-            for h in range(2):
-                yield from m.wait(f"B{h}", t)
-                acc(t, h, "dK")
-                yield
-            if t + STAGES_DKDV < n_t and plant != "early_release":
-                m.commit(f"YE{s}")
-            if more:
-                score(dp_cols, t + 1, "dP")
-                m.commit("DPF")
-            else:
-                m.commit("Done")
-            if plant == "early_release" and t + 1 + STAGES_DKDV < n_t:
-                m.commit(f"YE{(t + 1) % STAGES_DKDV}")
+        yc = tc = xi = 0
+        for i in range(len(seq)):
+            n = yield from ring.take(i)
+            if n < 0:
+                return
+            if n == 0:
+                continue
+            yield from m.wait("X", xi)
+            yield from m.wait(f"YF{yc % STAGES_DKDV}", yc // STAGES_DKDV)
+            score(s_cols, yc, tc, xi, "S")
+            m.commit("SF")
+            score(dp_cols, yc, tc, xi, "dP")
+            m.commit("DPF")
+            if n == 1:
+                m.commit("XE")
             yield
+            for t in range(n):
+                g, T = yc + t, tc + t
+                s = g % STAGES_DKDV
+                more = t + 1 < n
+                for h in range(2):
+                    yield from m.wait(f"A{h}", T)
+                    if t == 0 and h == 0 and xi > 0:
+                        yield from m.wait("AccE", xi - 1)
+                    accumulate(g, T, h, "dV", xi, t == 0 and h == 0)
+                    yield
+                if more:
+                    yield from m.wait(f"YF{(g + 1) % STAGES_DKDV}", (g + 1) // STAGES_DKDV)
+                    score(s_cols, g + 1, T + 1, xi, "S")
+                    m.commit("SF")
+                for h in range(2):
+                    yield from m.wait(f"B{h}", T)
+                    accumulate(g, T, h, "dK", xi, False)
+                    yield
+                if plant != "early_release":
+                    m.commit(f"YE{s}")
+                if more:
+                    score(dp_cols, g + 1, T + 1, xi, "dP")
+                    m.commit("DPF")
+                    if t + 1 == n - 1 or (plant == "xe_early" and t + 2 == n - 1):
+                        m.commit("XE")
+                else:
+                    m.commit("Done")
+                if plant == "early_release" and t + 1 < n:
+                    m.commit(f"YE{(g + 1) % STAGES_DKDV}")
+                yield
+            yc += n
+            tc += n
+            xi += 1
 
     def warp(h, w):
-        for t in range(n_t):
-            s = t % STAGES_DKDV
-            yield from m.wait(f"YF{s}", t // STAGES_DKDV)
-            ws_users[t] = ws_users.get(t, 0) + 1
-            yield from m.wait("SF", t)
-            if stage[s] != t:
-                raise ProtocolError("warp reads a stage without its tile")
-            state[(h, w, "S", t)] = True
-            if all(state.get((hh, ww, "S", t)) for hh in range(2) for ww in range(4)):
-                state[("S", t, "read")] = True
-            yield
-            state[(h, w, "P", t)] = True
-            wrote_p[(t, h)] = all(state.get((h, ww, "P", t)) for ww in range(4))
-            m.bars[f"A{h}"].arrive()
-            yield
-            yield from m.wait("DPF", t)
-            state[(h, w, "dP", t)] = True
-            if all(state.get((hh, ww, "dP", t)) for hh in range(2) for ww in range(4)):
-                state[("dP", t, "read")] = True
-            yield
-            wrote_ds[(t, h)] = all(state.get((h, ww, "dP", t)) for ww in range(4))
-            ws_users[t] -= 1
-            m.bars[f"B{h}"].arrive()
-            yield
-        yield from m.wait("Done", 0)
+        yc = tc = xi = 0
+        i = 0
+        n = yield from ring.take(0)
+        while n >= 0:
+            for t in range(n):
+                g, T = yc + t, tc + t
+                s = g % STAGES_DKDV
+                yield from m.wait(f"YF{s}", g // STAGES_DKDV)
+                ws_users[g] = ws_users.get(g, 0) + 1
+                yield from m.wait("SF", T if plant != "sf_parity" else T + 1)
+                if stage[s] != g or s_cols["T"] != T:
+                    raise ProtocolError("warp reads a stage or S^T without its tile")
+                state[(h, w, "S", T)] = True
+                if all(state.get((hh, ww, "S", T)) for hh in range(2) for ww in range(4)):
+                    state[("S", T, "read")] = True
+                yield
+                state[(h, w, "P", T)] = True
+                wrote_p[(T, h)] = all(state.get((h, ww, "P", T)) for ww in range(4))
+                m.bars[f"A{h}"].arrive()
+                yield
+                yield from m.wait("DPF", T)
+                if dp_cols["T"] != T:
+                    raise ProtocolError("warp reads dP^T without its tile")
+                state[(h, w, "dP", T)] = True
+                if all(state.get((hh, ww, "dP", T)) for hh in range(2) for ww in range(4)):
+                    state[("dP", T, "read")] = True
+                yield
+                wrote_ds[(T, h)] = all(state.get((h, ww, "dP", T)) for ww in range(4))
+                ws_users[g] -= 1
+                m.bars[f"B{h}"].arrive()
+                yield
+            nxt = yield from ring.take(i + 1)
+            if n > 0:
+                yield from m.wait("Done", xi)
+                if acc["item"] != xi or acc["last"] >= m.done:
+                    raise ProtocolError(f"warp reads item {xi}'s accumulators before its last product finished")
+                acc["read"][xi] = acc["read"].get(xi, 0) + 1
+                m.bars["AccE"].arrive()
+                xi += 1
+                yield
+            yc += n
+            tc += n
+            n = nxt
+            i += 1
 
     actors = {"loader": loader(), "mma": mma_warp()}
     for h in range(2):
@@ -167,111 +274,193 @@ def simulate_dkdv(n_t, seed, plant=None):
     m.run(actors)
 
 
-def simulate_dq(n_t, seed, plant=None):
+def simulate_dq(items, seed, plant=None):
+    """items: key-tile counts of the CTA's items, in order (0: no work)."""
     m = Model(seed)
-    m.bar("X")
+    seq = list(items) + [-1]
+    ring = ItemRing(m, seq, plant)
+    for name in ("X", "XE", "SF0", "SF1", "DPF", "Done"):
+        m.bar(name)
+    m.bar("AccE", 8)
     for s in range(K_STAGES_DQ):
         m.bar(f"KF{s}")
         m.bar(f"KE{s}")
     for s in range(V_STAGES_DQ):
         m.bar(f"VF{s}")
         m.bar(f"VE{s}")
-    for name in ("SF0", "SF1", "DPF", "Done"):
-        m.bar(name)
     for h in range(2):
         m.bar(f"B{h}", 4)
-    ring = {"K": [None] * K_STAGES_DQ, "V": [None] * V_STAGES_DQ}
+    rings = {"K": [None] * K_STAGES_DQ, "V": [None] * V_STAGES_DQ}
     landed = {"K": [False] * K_STAGES_DQ, "V": [False] * V_STAGES_DQ}
+    xbuf = {"item": None, "landed": False}
     readers = {}
-    sbuf = [None, None]  # tile held by S buffer 0 / 1
+    sbuf = [None, None]  # global score tile held by S buffer 0 / 1
+    dp = {"T": None}
+    acc = {"item": None, "last": -1, "read": {}}
     state = {}
 
+    def busy(key):
+        return any(i >= m.done for i in readers.get(key, []))
+
     def loader():
-        m.later(lambda: m.bars["X"].arrive())
-        for t in range(n_t):
-            for kind, n in (("K", K_STAGES_DQ), ("V", V_STAGES_DQ)):
-                s = t % n
-                if t >= n:
-                    yield from m.wait(f"{kind}E{s}", t // n - 1)
-                    if any(i >= m.done for i in readers.get((kind, t - n), [])):
-                        raise ProtocolError(f"{kind} stage {s} reloaded while tile {t - n} is read")
-                ring[kind][s], landed[kind][s] = t, False
+        cnt = {"K": 0, "V": 0}
+        xi = 0
+        for i, n in enumerate(seq):
+            yield from ring.publish(i)
+            yield
+            if n < 0:
+                return
+            if n == 0:
+                continue
+            if xi > 0 and plant != "x_early":
+                yield from m.wait("XE", xi - 1)
+            if busy(("X", xi - 1)):
+                raise ProtocolError(f"Q, dO of item {xi} loaded while item {xi - 1}'s products read theirs")
+            xbuf["item"], xbuf["landed"] = xi, False
 
-                def land(kind=kind, s=s):
-                    landed[kind][s] = True
-                    m.bars[f"{kind}F{s}"].arrive()
-                m.later(land)
-                yield
+            def land_x():
+                xbuf["landed"] = True
+                m.bars["X"].arrive()
+            m.later(land_x)
+            xi += 1
+            for _ in range(n):
+                for kind, ns in (("K", K_STAGES_DQ), ("V", V_STAGES_DQ)):
+                    g = cnt[kind]
+                    s = g % ns
+                    if g >= ns:
+                        yield from m.wait(f"{kind}E{s}", g // ns - 1)
+                        if busy((kind, g - ns)):
+                            raise ProtocolError(f"{kind} stage {s} reloaded while tile {g - ns} is read")
+                    rings[kind][s], landed[kind][s] = g, False
 
-    def use(kind, t, n):
-        s = t % n
-        if ring[kind][s] != t or not landed[kind][s]:
-            raise ProtocolError(f"MMA reads {kind} stage {s} without tile {t}")
+                    def land(kind=kind, s=s):
+                        landed[kind][s] = True
+                        m.bars[f"{kind}F{s}"].arrive()
+                    m.later(land)
+                    cnt[kind] += 1
+                    yield
+
+    def use(kind, g, ns, xi=None):
+        s = g % ns
+        if rings[kind][s] != g or not landed[kind][s]:
+            raise ProtocolError(f"MMA reads {kind} stage {s} without tile {g}")
         ids = [m.mma() for _ in range(8)]
-        readers.setdefault((kind, t), []).extend(ids)
+        readers.setdefault((kind, g), []).extend(ids)
+        if xi is not None:
+            if xbuf["item"] != xi or not xbuf["landed"]:
+                raise ProtocolError(f"MMA reads Q, dO without item {xi}'s")
+            readers.setdefault(("X", xi), []).extend(ids)
         return ids
 
-    def issue_s(t):
-        b = t & 1
-        if sbuf[b] is not None:
-            prev = sbuf[b]
-            if not state.get(("dS", prev, "written")) or not state.get(("dQ", prev)):
-                raise ProtocolError(f"S({t}) overwrites buffer {b} before dQ({prev}) is issued")
-        use("K", t, K_STAGES_DQ)
-        sbuf[b] = t
-        m.commit(f"SF{b}")
-
     def mma_warp():
-        yield from m.wait("X", 0)
-        yield from m.wait("KF0", 0)
-        issue_s(0)
-        yield from m.wait("VF0", 0)
-        use("V", 0, V_STAGES_DQ)
-        state[("dP", 0)] = True
-        m.commit("DPF")
-        if n_t > 1:
-            yield from m.wait("KF1", 0)
-            issue_s(1)
-        yield
-        for t in range(n_t):
-            for h in range(2):
-                yield from m.wait(f"B{h}", t)
-            state[("dS", t, "written")] = True
-            m.commit(f"VE{t % V_STAGES_DQ}")
-            if t + 1 < n_t:
-                u = t + 1
-                yield from m.wait(f"VF{u % V_STAGES_DQ}", u // V_STAGES_DQ)
-                use("V", u, V_STAGES_DQ)
-                state[("dP", u)] = True
-                m.commit("DPF")
-            if plant != "s_before_dq":
-                use("K", t, K_STAGES_DQ)  # dQ += dS(t) K_t
-                state[("dQ", t)] = True
-                m.commit(f"KE{t % K_STAGES_DQ}")
-            if t + 2 < n_t:
-                u = t + 2
-                yield from m.wait(f"KF{u % K_STAGES_DQ}", u // K_STAGES_DQ)
-                issue_s(u)
-            if plant == "s_before_dq":
-                use("K", t, K_STAGES_DQ)
-                state[("dQ", t)] = True
-                m.commit(f"KE{t % K_STAGES_DQ}")
-            if t == n_t - 1:
-                m.commit("Done")
+        kc = vc = tc = xi = 0
+
+        def issue_s(t):
+            T = tc + t
+            b = T & 1
+            if sbuf[b] is not None:
+                prev = sbuf[b]
+                if not state.get(("dS", prev, "written")) or not state.get(("dQ", prev)):
+                    raise ProtocolError(f"S({T}) overwrites buffer {b} before dQ({prev}) is issued")
+            use("K", kc + t, K_STAGES_DQ, xi)
+            sbuf[b] = T
+            m.commit(f"SF{b}")
+
+        def issue_dp(t):
+            T = tc + t
+            if dp["T"] is not None and not state.get(("dS", dp["T"], "written")):
+                raise ProtocolError(f"dP({T}) overwrites dP({dp['T']}) before both warpgroups read it")
+            use("V", vc + t, V_STAGES_DQ, xi)
+            dp["T"] = T
+            m.commit("DPF")
+
+        for i in range(len(seq)):
+            n = yield from ring.take(i)
+            if n < 0:
+                return
+            if n == 0:
+                continue
+            yield from m.wait("X", xi)
+            yield from m.wait(f"KF{kc % K_STAGES_DQ}", kc // K_STAGES_DQ)
+            issue_s(0)
+            yield from m.wait(f"VF{vc % V_STAGES_DQ}", vc // V_STAGES_DQ)
+            issue_dp(0)
+            if n == 1:
+                m.commit("XE")
+            if n > 1:
+                yield from m.wait(f"KF{(kc + 1) % K_STAGES_DQ}", (kc + 1) // K_STAGES_DQ)
+                issue_s(1)
             yield
+            for t in range(n):
+                T = tc + t
+                for h in range(2):
+                    yield from m.wait(f"B{h}", T)
+                state[("dS", T, "written")] = True
+                m.commit(f"VE{(vc + t) % V_STAGES_DQ}")
+                if t + 1 < n:
+                    u = vc + t + 1
+                    yield from m.wait(f"VF{u % V_STAGES_DQ}", u // V_STAGES_DQ)
+                    issue_dp(t + 1)
+                    if t + 1 == n - 1 and plant != "xe_early":
+                        m.commit("XE")
+                if t == 0 and xi > 0:
+                    yield from m.wait("AccE", xi - 1)
+                if t == 0 and xi > 0 and acc["read"].get(xi - 1, 0) < 8:
+                    raise ProtocolError(f"item {xi}'s first dQ overwrites item {xi - 1}'s before it is read")
+                if plant != "s_before_dq":
+                    ids = use("K", kc + t, K_STAGES_DQ)  # dQ += dS(t) K_t
+                    acc["item"], acc["last"] = xi, ids[-1]
+                    state[("dQ", T)] = True
+                    m.commit(f"KE{(kc + t) % K_STAGES_DQ}")
+                if t + 2 < n:
+                    u = kc + t + 2
+                    yield from m.wait(f"KF{u % K_STAGES_DQ}", u // K_STAGES_DQ)
+                    issue_s(t + 2)
+                if plant == "s_before_dq":
+                    ids = use("K", kc + t, K_STAGES_DQ)
+                    acc["item"], acc["last"] = xi, ids[-1]
+                    state[("dQ", T)] = True
+                    m.commit(f"KE{(kc + t) % K_STAGES_DQ}")
+                if plant == "xe_early" and t + 2 == n - 1:
+                    m.commit("XE")  # before S(n-1) and dP(n-1) are issued
+                if t == n - 1:
+                    m.commit("Done")
+                yield
+            kc += n
+            vc += n
+            tc += n
+            xi += 1
 
     def warp(h, w):
-        for t in range(n_t):
-            b = t & 1
-            yield from m.wait(f"SF{b}", t >> 1)
-            if sbuf[b] != t:
-                raise ProtocolError("warp reads an S buffer without its tile")
-            yield
-            yield from m.wait("DPF", t if plant != "dp_parity" else t + 1)
-            yield
-            m.bars[f"B{h}"].arrive()
-            yield
-        yield from m.wait("Done", 0)
+        tc = xi = 0
+        i = 0
+        n = yield from ring.take(0)
+        while n >= 0:
+            for t in range(n):
+                T = tc + t
+                b = T & 1
+                yield from m.wait(f"SF{b}", T >> 1)
+                if sbuf[b] != T:
+                    raise ProtocolError("warp reads an S buffer without its tile")
+                yield
+                yield from m.wait("DPF", T if plant != "dp_parity" else T + 1)
+                if dp["T"] != T:
+                    raise ProtocolError("warp reads dP without its tile")
+                yield
+                m.bars[f"B{h}"].arrive()
+                yield
+            nxt = yield from ring.take(i + 1)
+            if n > 0:
+                yield from m.wait("Done", xi)
+                if acc["item"] != xi or acc["last"] >= m.done:
+                    raise ProtocolError(f"warp reads item {xi}'s dQ before its last product finished")
+                acc["read"][xi] = acc["read"].get(xi, 0) + 1
+                m.bars["AccE"].arrive()
+                xi += 1
+                yield
+            tc += n
+            n = nxt
+            i += 1
 
     actors = {"loader": loader(), "mma": mma_warp()}
     for h in range(2):
@@ -280,30 +469,49 @@ def simulate_dq(n_t, seed, plant=None):
     m.run(actors)
 
 
-def _lengths(n, seed0):
+def _item_lists(n, seed0, max_items=6, max_tiles=7, zero_frac=0.2):
     r = random.Random(seed0)
-    return [(r.randint(1, 9), seed0 + i) for i in range(n)]
+    out = []
+    for i in range(n):
+        k = r.randint(1, max_items)
+        out.append(([0 if r.random() < zero_frac else r.randint(1, max_tiles) for _ in range(k)], seed0 + i))
+    return out
+
+
+def _planted_lists(plant, seed0):
+    """Item sequences that give a planted bug room to show: the item ring can
+    only run ahead through items without work; the rest need several tiles."""
+    if plant == "slot_early":
+        return [([0] * 4 + items, seed) for items, seed in _item_lists(300, seed0, zero_frac=0.6)]
+    return [([max(n, 3) for n in items] + [3], seed) for items, seed in _item_lists(300, seed0, zero_frac=0.0)]
 
 
 def test_dkdv_protocol_model_random_schedules():
-    for n_t, seed in _lengths(500, 0):
-        simulate_dkdv(n_t, seed)
+    for items, seed in _item_lists(400, 0):
+        simulate_dkdv(items, seed)
 
 
 def test_dq_protocol_model_random_schedules():
-    for n_t, seed in _lengths(500, 1000):
-        simulate_dq(n_t, seed)
+    for items, seed in _item_lists(400, 1000):
+        simulate_dq(items, seed)
 
 
-@pytest.mark.parametrize("plant", ["s_over_p", "early_release"])
+def test_single_items_and_edge_sequences():
+    for items in ([1], [2], [0], [0, 0], [1, 1, 1, 1], [0, 3, 0, 1], [9], [1, 9, 1]):
+        for seed in range(20):
+            simulate_dkdv(items, seed)
+            simulate_dq(items, seed)
+
+
+@pytest.mark.parametrize("plant", ["early_release", "x_early", "xe_early", "slot_early", "sf_parity"])
 def test_dkdv_protocol_model_catches_planted_bugs(plant):
     with pytest.raises(ProtocolError):
-        for n_t, seed in _lengths(300, 0):
-            simulate_dkdv(max(n_t, 3), seed, plant=plant)
+        for items, seed in _planted_lists(plant, 0):
+            simulate_dkdv(items, seed, plant=plant)
 
 
-@pytest.mark.parametrize("plant", ["s_before_dq", "dp_parity"])
+@pytest.mark.parametrize("plant", ["s_before_dq", "dp_parity", "x_early", "xe_early", "slot_early"])
 def test_dq_protocol_model_catches_planted_bugs(plant):
     with pytest.raises(ProtocolError):
-        for n_t, seed in _lengths(300, 1000):
-            simulate_dq(max(n_t, 3), seed, plant=plant)
+        for items, seed in _planted_lists(plant, 1000):
+            simulate_dq(items, seed, plant=plant)
