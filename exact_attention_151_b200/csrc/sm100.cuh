@@ -227,25 +227,6 @@ __device__ __forceinline__ void bulk_load_elect(uint32_t dst, const void* src, u
       : "memory");
 }
 
-// 64 bytes (32 16-bit values, packed in pairs) to global memory: two 32-byte
-// stores when `wide` (dst 32-byte aligned), else four 16-byte ones. When the
-// 32 lanes of a warp write 32 different rows, each store instruction costs
-// the L1 one pass per row, so the wide form halves the passes.
-__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&pk)[16], bool wide) {
-  if (wide) {
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(static_cast<char*>(dst) + 32 * k),
-                   "r"(pk[8 * k]), "r"(pk[8 * k + 1]), "r"(pk[8 * k + 2]), "r"(pk[8 * k + 3]), "r"(pk[8 * k + 4]),
-                   "r"(pk[8 * k + 5]), "r"(pk[8 * k + 6]), "r"(pk[8 * k + 7])
-                   : "memory");
-  } else {
-    uint4* d = static_cast<uint4*>(dst);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) d[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-  }
-}
-
 // Tiled TMA store shared -> global of one box at (c0, c1, c2), issued by one
 // thread, in a bulk group; shared-memory writes by other threads must be made
 // visible to the async proxy first (fence_proxy_async_smem, then a barrier).
