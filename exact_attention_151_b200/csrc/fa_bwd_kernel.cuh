@@ -53,23 +53,28 @@ struct Cfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kSlabBytes = 128 * 128;
   static constexpr int kTileBytes = kHalves * kSlabBytes;
-  static constexpr int kStages = 2;
+  // D = 64: TMEM holds two S^T buffers beside dP^T and the two 64-column
+  // accumulators, so S^T(t+2) is issued as soon as dV(t) has read P^T(t); a
+  // third ring stage keeps its operands loaded by then.
+  static constexpr bool kDoubleS = D == 64;
+  static constexpr int kSBufs = kDoubleS ? 2 : 1;
+  static constexpr int kStages = kDoubleS ? 3 : 2;
   static constexpr int kXOff = 0;                              // fixed operands X1, X2
   static constexpr int kYOff = kXOff + 2 * kTileBytes;          // ring of (Y1, Y2) pairs
   static constexpr int kBarOff = kYOff + kStages * 2 * kTileBytes;
   static constexpr int kBarX = 0;
-  static constexpr int kBarYFull = 1;                 // [kStages]
-  static constexpr int kBarYEmpty = 1 + kStages;      // [kStages]
-  static constexpr int kBarSFull = 1 + 2 * kStages;   // scores S (or S^T) in TMEM
-  static constexpr int kBarDPFull = kBarSFull + 1;    // dP (or dP^T) in TMEM
-  static constexpr int kBarA = kBarDPFull + 1;        // [2] phase A of warpgroup h done (128 arrivals)
-  static constexpr int kBarB = kBarA + 2;             // [2] phase B of warpgroup h done (128 arrivals)
-  static constexpr int kBarDone = kBarB + 2;          // last accumulating MMA of an item finished
+  static constexpr int kBarYFull = 1;                       // [kStages]
+  static constexpr int kBarYEmpty = 1 + kStages;            // [kStages]
+  static constexpr int kBarSFull = 1 + 2 * kStages;         // [kSBufs] scores S^T of buffer b in TMEM
+  static constexpr int kBarDPFull = kBarSFull + kSBufs;     // dP^T in TMEM
+  static constexpr int kBarA = kBarDPFull + 1;              // [kSBufs][2] phase A of warpgroup h on buffer b done (128 arrivals)
+  static constexpr int kBarB = kBarA + 2 * kSBufs;          // [2] phase B of warpgroup h done (128 arrivals)
+  static constexpr int kBarDone = kBarB + 2;                // last accumulating MMA of an item finished
   static constexpr int kBarDrain = kBarDone + 1;
-  static constexpr int kBarXEmpty = kBarDrain + 1;    // last MMA reading X1, X2 of an item finished
-  static constexpr int kBarAccEmpty = kBarXEmpty + 1; // accumulators read out (256 arrivals)
-  static constexpr int kBarItemFull = kBarAccEmpty + 1;   // [2] work-item slot written
-  static constexpr int kBarItemEmpty = kBarItemFull + 2;  // [2] work-item slot read (kItemReaders arrivals)
+  static constexpr int kBarXEmpty = kBarDrain + 1;          // last MMA reading X1, X2 of an item finished
+  static constexpr int kBarAccEmpty = kBarXEmpty + 1;       // accumulators read out (256 arrivals)
+  static constexpr int kBarItemFull = kBarAccEmpty + 1;     // [2] work-item slot written
+  static constexpr int kBarItemEmpty = kBarItemFull + 2;    // [2] work-item slot read (kItemReaders arrivals)
   static constexpr int kNumBars = kBarItemEmpty + 2;
   static constexpr int kWsOff = kBarOff + 256;        // key side, per stage: -LSE log2(e) and -D of the 128 queries
   static constexpr int kWsBytes = 2 * 128 * 4;
@@ -77,9 +82,10 @@ struct Cfg {
   static_assert(kNumBars * 8 <= 256, "barrier area");
   static constexpr int kSmemBytes = kMiscOff + 32 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  // TMEM columns: S^T, dP^T, accumulators acc0 = dK, acc1 = dV.
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
-  static_assert(256 + 2 * D <= 512, "TMEM budget");
+  // TMEM columns: S^T buffer b at col_s(b), dP^T, accumulators acc0 = dK, acc1 = dV.
+  __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * static_cast<uint32_t>(b); }
+  static constexpr uint32_t kColDP = 128 * kSBufs, kColAcc0 = kColDP + 128, kColAcc1 = kColAcc0 + D;
+  static_assert(kColAcc1 + D <= 512, "TMEM budget");
 };
 
 // Shapes: q, o, dO, dQ [B, Nq, Hq, D]; k, v, dK, dV [B, Nk, Hkv, D] (dense), or
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_varlen_kernel(const uint16_t*
 }
 
 // Phase A for one thread's half row: p = 2^(s c + nl) for the 64 scores of
-// TMEM columns kColS + 64h .. (two 32-column chunks). nl is -LSE log2(e):
+// TMEM columns t_s .. t_s + 63 of the score buffer (two 32-column chunks). nl is -LSE log2(e):
 // per row (query side, `nl_row`) or per column from shared memory (key side,
 // `nl_col`). MASKED tiles (causal tiles the diagonal cuts, key j visible to
 // query i iff j <= i + delta, or the ragged tail of the keys) zero the
@@ -496,10 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarYFull + s), 1);
       mbar_init(bar(C::kBarYEmpty + s), 1);
     }
-    mbar_init(bar(C::kBarSFull), 1);
+    for (int b = 0; b < C::kSBufs; ++b) {
+      mbar_init(bar(C::kBarSFull + b), 1);
+      for (int h = 0; h < 2; ++h) mbar_init(bar(C::kBarA + 2 * b + h), 128);
+    }
     mbar_init(bar(C::kBarDPFull), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(C::kBarA + i), 128);
       mbar_init(bar(C::kBarB + i), 128);
       mbar_init(bar(C::kBarItemFull + i), 1);
       mbar_init(bar(C::kBarItemEmpty + i), kItemReaders);
@@ -620,34 +628,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = warp_wait_bar(bar(C::kBarX), static_cast<uint32_t>(xi & 1), wc) &&
            warp_wait_bar(bar(C::kBarYFull + ystage(0)), yphase(0), wc);
       if (!ok) break;
+      // score tile T (counted across items) goes to S^T buffer T % kSBufs
+      auto sbuf = [&](int t) { return (tc + t) % C::kSBufs; };
+      auto issue_s = [&](int t) {
+        issue_score(0, ystage(t), C::col_s(sbuf(t)));
+        mma_commit_elect(bar(C::kBarSFull + sbuf(t)));
+      };
       tc_fence_after();
-      issue_score(0, ystage(0), C::kColS);
-      mma_commit_elect(bar(C::kBarSFull));
+      issue_s(0);
       issue_score(1, ystage(0), C::kColDP);
       mma_commit_elect(bar(C::kBarDPFull));
       if (n == 1) mma_commit_elect(bar(C::kBarXEmpty));  // K, V of this item: last readers issued
+      if (C::kDoubleS && n > 1) {
+        ok = warp_wait_bar(bar(C::kBarYFull + ystage(1)), yphase(1), wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(1);
+      }
       for (int t = 0; ok && t < n; ++t) {
         const uint32_t ph = static_cast<uint32_t>((tc + t) & 1);
+        const uint32_t pa = static_cast<uint32_t>(((tc + t) / C::kSBufs) & 1);  // phase of this tile's buffer
         const bool more = t + 1 < n;
         // dV += P^T dO per half as each warpgroup publishes its P^T; the first
         // one of an item waits until the previous item's accumulators are read out
         for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = warp_wait_bar(bar(C::kBarA + hf), ph, wc);
+          ok = warp_wait_bar(bar(C::kBarA + 2 * sbuf(t) + hf), pa, wc);
           if (ok && t == 0 && hf == 0 && xi > 0)
             ok = warp_wait_bar(bar(C::kBarAccEmpty), static_cast<uint32_t>((xi - 1) & 1), wc);
           if (ok) {
             tc_fence_after();
-            issue_acc(C::kColAcc1, C::kColS + 64 * hf, 1, ystage(t), hf, t == 0 && hf == 0);
+            issue_acc(C::kColAcc1, C::col_s(sbuf(t)) + 64 * hf, 1, ystage(t), hf, t == 0 && hf == 0);
           }
         }
         if (!ok) break;
-        // S^T of the next tile (its P^T columns are free once dV has read them: in-order)
-        if (more) {
+        // one buffer: S^T of the next tile (its P^T columns are free once dV has read them: in-order)
+        if (!C::kDoubleS && more) {
           ok = warp_wait_bar(bar(C::kBarYFull + ystage(t + 1)), yphase(t + 1), wc);
           if (!ok) break;
           tc_fence_after();
-          issue_score(0, ystage(t + 1), C::kColS);
-          mma_commit_elect(bar(C::kBarSFull));
+          issue_s(t + 1);
         }
         // dK += dS^T Q per half
         for (int hf = 0; hf < 2 && ok; ++hf) {
@@ -664,6 +683,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_score(1, ystage(t + 1), C::kColDP);
           mma_commit_elect(bar(C::kBarDPFull));
           if (t + 1 == n - 1) mma_commit_elect(bar(C::kBarXEmpty));
+          // two buffers: S^T two tiles ahead, into the buffer whose P^T dV(t) has read (in order)
+          if (C::kDoubleS && t + 2 < n) {
+            ok = warp_wait_bar(bar(C::kBarYFull + ystage(t + 2)), yphase(t + 2), wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t + 2);
+          }
         } else {
           mma_commit_elect(bar(C::kBarDone));
         }
@@ -684,7 +710,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const float c = prm.scale_log2;
     const float nl_row = 0.f, nd_row = 0.f;  // per-column values on this side
-    const uint32_t t_s = tmem + lane_base + C::kColS + 64 * wg;
     const uint32_t t_dp = tmem + lane_base + C::kColDP + 64 * wg;
     const uint32_t t_ds = t_dp;  // dS^T pairs over the first half of this half of dP^T
     int yc = 0, tc = 0, xi = 0;
@@ -702,6 +727,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = yc + t;
         const int s = g % C::kStages;
         const uint32_t ph = static_cast<uint32_t>((tc + t) & 1);
+        const int sb = (tc + t) % C::kSBufs;                                   // this tile's S^T buffer
+        const uint32_t pa = static_cast<uint32_t>(((tc + t) / C::kSBufs) & 1);  // and that buffer's phase
+        const uint32_t t_s = tmem + lane_base + C::col_s(sb) + 64 * wg;
         const int cbase = (it.t_first + t % it.per_head) * kTile;  // first query (column) of this pair's tile
         const int first_col = cbase + 64 * wg;
         // this tile's -LSE log2(e) and -D for the warpgroup's 64 query columns,
@@ -713,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool masked = (causal && it.tile * kTile + kTile - 1 > cbase + it.sq.delta) || cbase + kTile > it.sq.nq;
         ok = warp_wait_bar(bar(C::kBarYFull + s), static_cast<uint32_t>((g / C::kStages) & 1), wc);
         if (!ok) break;
-        ok = warp_wait_bar(bar(C::kBarSFull), ph, wc);
+        ok = warp_wait_bar(bar(C::kBarSFull + sb), pa, wc);
         if (!ok) break;
         tc_fence_after();
         float p[64];
@@ -724,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(C::kBarA + wg));
+        mbar_arrive(bar(C::kBarA + 2 * sb + wg));
         ok = warp_wait_bar(bar(C::kBarDPFull), ph, wc);
         if (!ok) break;
         tc_fence_after();

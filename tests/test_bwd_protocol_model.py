@@ -20,7 +20,12 @@ previous item's out (AccEmpty).
 dK/dV: per item, the MMA warp issues S^T(0) and dP^T(0), then per tile t:
 dV += P^T dO per half (after that half's phase A), S^T(t+1) over the P^T
 columns, dK += dS^T Q per half (after phase B), the stage release, and dP^T(t+1)
-over the dS^T columns (or the item's final commit).
+over the dS^T columns (or the item's final commit). At D = 64 (TMEM has room)
+two S^T buffers: S^T(0) and S^T(1) up front, and S^T(t+2) right after
+dP^T(t+1), into the buffer dV(t) has just read, with a three-stage ring; the
+phase-A barriers are then per buffer too (with one, a warpgroup can finish
+phase A of two tiles before the MMA warp waits for the first: two phases
+ahead, which a parity wait misreads; planted as "db_one_a").
 
 dQ: K_t into a 3-stage ring, V_t into a 2-stage ring. Per item the MMA warp
 issues S(0), dP(0), S(1), then per tile t: after both warpgroups' phase B,
@@ -76,26 +81,35 @@ class ItemRing:
         return n
 
 
-def simulate_dkdv(items, seed, plant=None):
-    """items: streamed-tile counts of the CTA's items, in order (0: no work)."""
+def simulate_dkdv(items, seed, plant=None, db=False):
+    """items: streamed-tile counts of the CTA's items, in order (0: no work).
+    db: the D = 64 form, with two S^T buffers (one score barrier each) and a
+    three-stage ring; S^T(t+2) is issued right after dP^T(t+1), into the buffer
+    whose P^T dV(t) has just read."""
     m = Model(seed)
     seq = list(items) + [-1]
     ring = ItemRing(m, seq, plant)
-    for name in ("X", "XE", "SF", "DPF", "Done", "Drain"):
+    n_stages = 3 if db else STAGES_DKDV
+    n_sbuf = 2 if db else 1
+    for name in ("X", "XE", "DPF", "Done", "Drain"):
         m.bar(name)
+    for b in range(n_sbuf):
+        m.bar(f"SF{b}")
     m.bar("AccE", 8)
-    for s in range(STAGES_DKDV):
+    for s in range(n_stages):
         m.bar(f"YF{s}")
         m.bar(f"YE{s}")
     for h in range(2):
-        m.bar(f"A{h}", 4)
+        for b in range(n_sbuf):  # double-buffered: one phase-A barrier per S^T buffer
+            m.bar(f"A{b}{h}", 4)
         m.bar(f"B{h}", 4)
-    stage = [None] * STAGES_DKDV   # global streamed tile held
-    landed = [False] * STAGES_DKDV
+    stage = [None] * n_stages   # global streamed tile held
+    landed = [False] * n_stages
     xbuf = {"item": None, "landed": False}
     readers = {}     # ("Y", g) / ("X", xi) -> MMA ids reading it
     ws_users = {}    # g -> warps still reading the stage's -LSE / -D rows
-    s_cols, dp_cols = {"T": None}, {"T": None}
+    s_cols = [{"T": None} for _ in range(n_sbuf)]
+    dp_cols = {"T": None}
     wrote_p, wrote_ds = {}, {}
     acc = {"item": None, "last": -1, "read": {}}  # item accumulating; last MMA id into it; warps that read item xi
     state = {}
@@ -124,13 +138,13 @@ def simulate_dkdv(items, seed, plant=None):
             m.later(land_x)
             xi += 1
             for _ in range(n):
-                s = yc % STAGES_DKDV
-                if yc >= STAGES_DKDV:
-                    yield from m.wait(f"YE{s}", yc // STAGES_DKDV - 1)
-                    if busy(("Y", yc - STAGES_DKDV)):
-                        raise ProtocolError(f"stage {s} reloaded while an MMA reads tile {yc - STAGES_DKDV}")
-                    if ws_users.get(yc - STAGES_DKDV):
-                        raise ProtocolError(f"stage {s} reloaded while a warp reads tile {yc - STAGES_DKDV}'s rows")
+                s = yc % n_stages
+                if yc >= n_stages:
+                    yield from m.wait(f"YE{s}", yc // n_stages - 1)
+                    if busy(("Y", yc - n_stages)):
+                        raise ProtocolError(f"stage {s} reloaded while an MMA reads tile {yc - n_stages}")
+                    if ws_users.get(yc - n_stages):
+                        raise ProtocolError(f"stage {s} reloaded while a warp reads tile {yc - n_stages}'s rows")
                 stage[s], landed[s] = yc, False
 
                 def land(s=s):
@@ -141,7 +155,7 @@ def simulate_dkdv(items, seed, plant=None):
                 yield
 
     def score(cols, g, T, xi, what):
-        s = g % STAGES_DKDV
+        s = g % n_stages
         if stage[s] != g or not landed[s]:
             raise ProtocolError(f"{what}({T}) reads a stage without tile {g}")
         if xbuf["item"] != xi or not xbuf["landed"]:
@@ -159,6 +173,11 @@ def simulate_dkdv(items, seed, plant=None):
         readers.setdefault(("Y", g), []).extend(ids)
         readers.setdefault(("X", xi), []).extend(ids)
         cols["T"] = T
+
+    def issue_s(g, T, xi):
+        b = T % n_sbuf
+        score(s_cols[b], g, T, xi, "S")
+        m.commit(f"SF{b}")
 
     def accumulate(g, T, h, kind, xi, first):
         if not (wrote_p if kind == "dV" else wrote_ds).get((T, h)):
@@ -179,28 +198,33 @@ def simulate_dkdv(items, seed, plant=None):
             if n == 0:
                 continue
             yield from m.wait("X", xi)
-            yield from m.wait(f"YF{yc % STAGES_DKDV}", yc // STAGES_DKDV)
-            score(s_cols, yc, tc, xi, "S")
-            m.commit("SF")
+            yield from m.wait(f"YF{yc % n_stages}", yc // n_stages)
+            issue_s(yc, tc, xi)
             score(dp_cols, yc, tc, xi, "dP")
             m.commit("DPF")
             if n == 1:
                 m.commit("XE")
+            if db and n > 1:
+                yield from m.wait(f"YF{(yc + 1) % n_stages}", (yc + 1) // n_stages)
+                issue_s(yc + 1, tc + 1, xi)
             yield
             for t in range(n):
                 g, T = yc + t, tc + t
-                s = g % STAGES_DKDV
+                s = g % n_stages
                 more = t + 1 < n
+                if db and plant == "db_s_early" and t + 2 < n:
+                    yield from m.wait(f"YF{(g + 2) % n_stages}", (g + 2) // n_stages)
+                    issue_s(g + 2, T + 2, xi)  # before dV(t) has read P^T(t) from that buffer
                 for h in range(2):
-                    yield from m.wait(f"A{h}", T)
+                    a_k = T // n_sbuf if plant != "db_one_a" else T
+                    yield from m.wait(f"A{T % n_sbuf if plant != 'db_one_a' else 0}{h}", a_k)
                     if t == 0 and h == 0 and xi > 0:
                         yield from m.wait("AccE", xi - 1)
                     accumulate(g, T, h, "dV", xi, t == 0 and h == 0)
                     yield
-                if more:
-                    yield from m.wait(f"YF{(g + 1) % STAGES_DKDV}", (g + 1) // STAGES_DKDV)
-                    score(s_cols, g + 1, T + 1, xi, "S")
-                    m.commit("SF")
+                if more and not db:
+                    yield from m.wait(f"YF{(g + 1) % n_stages}", (g + 1) // n_stages)
+                    issue_s(g + 1, T + 1, xi)
                 for h in range(2):
                     yield from m.wait(f"B{h}", T)
                     accumulate(g, T, h, "dK", xi, False)
@@ -212,10 +236,13 @@ def simulate_dkdv(items, seed, plant=None):
                     m.commit("DPF")
                     if t + 1 == n - 1 or (plant == "xe_early" and t + 2 == n - 1):
                         m.commit("XE")
+                    if db and plant != "db_s_early" and t + 2 < n:
+                        yield from m.wait(f"YF{(g + 2) % n_stages}", (g + 2) // n_stages)
+                        issue_s(g + 2, T + 2, xi)
                 else:
                     m.commit("Done")
                 if plant == "early_release" and t + 1 < n:
-                    m.commit(f"YE{(g + 1) % STAGES_DKDV}")
+                    m.commit(f"YE{(g + 1) % n_stages}")
                 yield
             yc += n
             tc += n
@@ -228,11 +255,13 @@ def simulate_dkdv(items, seed, plant=None):
         while n >= 0:
             for t in range(n):
                 g, T = yc + t, tc + t
-                s = g % STAGES_DKDV
-                yield from m.wait(f"YF{s}", g // STAGES_DKDV)
+                s = g % n_stages
+                b = T % n_sbuf
+                yield from m.wait(f"YF{s}", g // n_stages)
                 ws_users[g] = ws_users.get(g, 0) + 1
-                yield from m.wait("SF", T if plant != "sf_parity" else T + 1)
-                if stage[s] != g or s_cols["T"] != T:
+                k = T // n_sbuf
+                yield from m.wait(f"SF{b}", k if plant != "sf_parity" else k + 1)
+                if stage[s] != g or s_cols[b]["T"] != T:
                     raise ProtocolError("warp reads a stage or S^T without its tile")
                 state[(h, w, "S", T)] = True
                 if all(state.get((hh, ww, "S", T)) for hh in range(2) for ww in range(4)):
@@ -240,7 +269,7 @@ def simulate_dkdv(items, seed, plant=None):
                 yield
                 state[(h, w, "P", T)] = True
                 wrote_p[(T, h)] = all(state.get((h, ww, "P", T)) for ww in range(4))
-                m.bars[f"A{h}"].arrive()
+                m.bars[f"A{b if plant != 'db_one_a' else 0}{h}"].arrive()
                 yield
                 yield from m.wait("DPF", T)
                 if dp_cols["T"] != T:
@@ -491,15 +520,21 @@ def test_dkdv_protocol_model_random_schedules():
         simulate_dkdv(items, seed)
 
 
+def test_dkdv_double_buffered_protocol_model_random_schedules():
+    for items, seed in _item_lists(400, 500):
+        simulate_dkdv(items, seed, db=True)
+
+
 def test_dq_protocol_model_random_schedules():
     for items, seed in _item_lists(400, 1000):
         simulate_dq(items, seed)
 
 
 def test_single_items_and_edge_sequences():
-    for items in ([1], [2], [0], [0, 0], [1, 1, 1, 1], [0, 3, 0, 1], [9], [1, 9, 1]):
+    for items in ([1], [2], [0], [0, 0], [1, 1, 1, 1], [0, 3, 0, 1], [9], [1, 9, 1], [2, 2, 3]):
         for seed in range(20):
             simulate_dkdv(items, seed)
+            simulate_dkdv(items, seed, db=True)
             simulate_dq(items, seed)
 
 
@@ -508,6 +543,14 @@ def test_dkdv_protocol_model_catches_planted_bugs(plant):
     with pytest.raises(ProtocolError):
         for items, seed in _planted_lists(plant, 0):
             simulate_dkdv(items, seed, plant=plant)
+
+
+@pytest.mark.parametrize("plant", ["early_release", "x_early", "xe_early", "slot_early", "sf_parity", "db_s_early",
+                                   "db_one_a"])
+def test_dkdv_double_buffered_protocol_model_catches_planted_bugs(plant):
+    with pytest.raises(ProtocolError):
+        for items, seed in _planted_lists(plant, 700):
+            simulate_dkdv(items, seed, plant=plant, db=True)
 
 
 @pytest.mark.parametrize("plant", ["s_before_dq", "dp_parity", "x_early", "xe_early", "slot_early"])
