@@ -166,51 +166,75 @@ __device__ __forceinline__ void store_row64(void* dst, const uint32_t (&pk)[16],
 }
 
 // -D_i and -LSE_i log2(e) per row into the tile-padded workspace (negated:
-// the kernels add them). Blocks below n_real_blocks read O and dO in memory
-// order ([B, N, H, D] rows, D / 8 threads per row, 16-byte loads); the rest
-// fill the pad rows (D = 0, LSE = +inf).
+// the kernels add them); pad rows get D = 0, LSE = +inf (weights exactly 0).
+// Streaming work, bound by reading O and dO once: a grid of a few blocks per
+// SM strides over items of kPrepRowsPerIter consecutive rows i of one (b, h);
+// D / 8 threads read a row's 16-byte pieces (each row is D * 2 contiguous
+// bytes of [B, N, H, D]) and every thread keeps kPrepUnroll rows' loads in
+// flight. Consecutive i keep the LSE reads and the workspace writes contiguous.
+constexpr int kPrepUnroll = 4;
+template <int D>
+__host__ __device__ constexpr int prep_rows_per_iter() {
+  return 8 * (32 / (D / 8)) * kPrepUnroll;  // 8 warps, 32 / (D / 8) rows per warp, kPrepUnroll deep
+}
+
 template <int D, bool FP16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __restrict__ o,
                                                           const uint16_t* __restrict__ dout,
                                                           const float* __restrict__ lse, float* __restrict__ ws_d,
                                                           float* __restrict__ ws_l, int B, int N, int H, int Npad,
-                                                          unsigned n_real_blocks, int* __restrict__ sched) {
+                                                          int* __restrict__ sched) {
   constexpr int kLanes = D / 8;                 // threads per row
-  constexpr int kRowsPerBlock = 256 / kLanes;
+  constexpr int kRowsPerWarp = 32 / kLanes;
+  constexpr int kRows = prep_rows_per_iter<D>();
   if (blockIdx.x == 0 && threadIdx.x < 2) sched[threadIdx.x] = 0;  // the gradient kernels' work-item counters
-  const int64_t n_rows = static_cast<int64_t>(B) * N * H;
-  if (blockIdx.x < n_real_blocks) {
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanes;  // (b N + i) H + h
-    const int sub = threadIdx.x % kLanes;
-    const bool valid = row < n_rows;
-    float acc = 0.f;
-    if (valid) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
-      const uint4 y = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
-      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, sub = lane % kLanes;
+  const int chunks = (N + kRows - 1) / kRows;
+  const int64_t n_items = static_cast<int64_t>(B) * H * chunks;
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t bh = item / chunks;
+    const int c = static_cast<int>(item - bh * chunks);
+    const int64_t b = bh / H;
+    const int h = static_cast<int>(bh - b * H);
+    const int i0 = c * kRows + warp * kRowsPerWarp * kPrepUnroll + lane / kLanes;
+    uint4 x[kPrepUnroll], y[kPrepUnroll];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 a = unpack2<FP16>(xs[k]);
-        const float2 c = unpack2<FP16>(ys[k]);
-        acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      const int i = i0 + u * kRowsPerWarp;
+      x[u] = make_uint4(0u, 0u, 0u, 0u);
+      y[u] = x[u];
+      if (i < N) {
+        const int64_t row = (b * N + i) * H + h;
+        x[u] = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
+        y[u] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
       }
     }
 #pragma unroll
-    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (valid && sub == 0) {
-      const int h = static_cast<int>(row % H);
-      const int64_t bi = row / H;
-      const int i = static_cast<int>(bi % N);
-      const int64_t bh = (bi / N) * H + h;
-      ws_d[bh * Npad + i] = -acc;
-      // a row that sees no key has LSE = -inf: its weights are 0, not exp(+inf)
-      const float l = lse[bh * N + i];
-      ws_l[bh * Npad + i] = l == -INFINITY ? -INFINITY : -l * 1.44269504088896340736f;
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      const int i = i0 + u * kRowsPerWarp;
+      const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w}, ys[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 a = unpack2<FP16>(xs[k]);
+        const float2 cc = unpack2<FP16>(ys[k]);
+        acc = fmaf(a.x, cc.x, fmaf(a.y, cc.y, acc));
+      }
+#pragma unroll
+      for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (i < N && sub == 0) {
+        ws_d[bh * Npad + i] = -acc;
+        // a row that sees no key has LSE = -inf: its weights are 0, not exp(+inf)
+        const float l = lse[bh * N + i];
+        ws_l[bh * Npad + i] = l == -INFINITY ? -INFINITY : -l * 1.44269504088896340736f;
+      }
     }
-  } else {
-    const int pad = Npad - N;
-    const int64_t p = static_cast<int64_t>(blockIdx.x - n_real_blocks) * 256 + threadIdx.x;
-    if (pad > 0 && p < static_cast<int64_t>(B) * H * pad) {
+  }
+  const int pad = Npad - N;
+  if (pad > 0) {
+    const int64_t n_pad = static_cast<int64_t>(B) * H * pad;
+    for (int64_t p = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; p < n_pad;
+         p += static_cast<int64_t>(gridDim.x) * 256) {
       const int64_t idx = (p / pad) * Npad + N + p % pad;
       ws_d[idx] = 0.f;
       ws_l[idx] = -INFINITY;

@@ -409,10 +409,12 @@ fa_status bwd_run(int dev, const void* q, const void* k, const void* v, const vo
           static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(tq_rows), static_cast<int>(npad),
           static_cast<unsigned>(real_blocks), sched);
     } else {
-      bwd::fa_bwd_prep_kernel<D, FP16><<<grid, 256, 0, stream>>>(
+      // a few blocks per SM striding over (b, h, rows) items
+      const int64_t items = BHq * ((Nq + bwd::prep_rows_per_iter<D>() - 1) / bwd::prep_rows_per_iter<D>());
+      const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(items, 8 * static_cast<int64_t>(device_sm_count(dev))));
+      bwd::fa_bwd_prep_kernel<D, FP16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
           static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, ws_d, ws_l, static_cast<int>(B),
-          static_cast<int>(Nq), static_cast<int>(Hq), static_cast<int>(npad), static_cast<unsigned>(real_blocks),
-          sched);
+          static_cast<int>(Nq), static_cast<int>(Hq), static_cast<int>(npad), sched);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
