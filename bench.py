@@ -459,6 +459,9 @@ def main():
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--shard", action="store_true",
                     help="split one workload over the ranks (batch or heads) and all-gather O and LSE each step")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="forward: launch every timed step through the Python API instead of replaying a CUDA graph "
+                         "of one step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -621,6 +624,22 @@ def run_forward(args, w, dev, world, rank):
         step()
     if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
         raise RuntimeError("device status word reports a timeout during warm-up")
+    # One step captured as a CUDA graph (the same kernel launches with the same
+    # buffers), replayed once per timed step, so that the host's per-call
+    # Python and argument marshalling stay off the device timeline; short steps
+    # (decode, the small config) are otherwise bound by the host.
+    graph = None
+    if not args.no_graph and not shard:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        if fa.status_sync(stream.cuda_stream) != fa.FA_OK:
+            raise RuntimeError("device status word reports a timeout in the captured step")
+
+        def step():  # noqa: F811
+            graph.replay()
 
     # ---- timed region: exactly K steps, per-step events on the launching stream
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -677,6 +696,8 @@ def run_forward(args, w, dev, world, rank):
         # the kernel's roofline: tensor-bound above the ridge of the measured peaks
         ridge = peak * 1e12 / (measured_hbm() * 1e9)
         cfg = workload_config(w)
+        cfg["launch"] = ("a CUDA graph of one step (the same kernel launches), replayed per timed step" if graph is not None
+                         else "one Python API call per timed step")
         if shard:
             cfg["parallelism"] = (f"shard over {'batch' if shard[0].axis == 0 else 'heads'} on {world} rank(s) "
                                   "+ NCCL all-gather of O and LSE (inside each step)")
