@@ -8,7 +8,7 @@ report a failure through the status word (a debugging aid; slower).
 
 The library is compiled for sm_100a only (tcgen05 / TMA / Tensor Memory), with
 the CUDA runtime linked statically so the shared object loads on a machine
-without a GPU (symbol checks) and on the GPU machine alike.
+without a GPU (symbol checks) and on a B200 host alike.
 """
 
 from __future__ import annotations
