@@ -590,10 +590,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       // Both halves of PV_i(j) with the V item u: each waits for its half of P.
-      auto issue_pv = [&](int i, int j, int u, bool split) -> bool {
+      // V is waited for first (with need_v; false when this warp has already
+      // observed V item u): it is normally resident by now, and P, which is
+      // not, then ends the wait with nothing left to check behind it.
+      auto issue_pv = [&](int i, int j, int u, bool split, bool need_v) -> bool {
         const int sv = u % C::kVStages;
-        if (!warp_wait_bar(bar(C::kBarPFull + 2 * i), static_cast<uint32_t>(j & 1), wc) ||
-            !warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((u / C::kVStages) & 1), wc))
+        if ((need_v && !warp_wait_bar(bar(C::kBarVFull + sv), static_cast<uint32_t>((u / C::kVStages) & 1), wc)) ||
+            !warp_wait_bar(bar(C::kBarPFull + 2 * i), static_cast<uint32_t>(j & 1), wc))
           return false;
         tc_fence_after();
         issue_pv_half(i, j, sv, split, 0);
@@ -611,19 +614,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return true;
       };
+      // Every wait between two MMA groups leaves the tensor pipe idle while it
+      // runs, even one already satisfied (an mbarrier poll with its warp vote
+      // takes longer than the one MMA the pipe still holds). So, unpaired,
+      // the waits that are normally satisfied are taken where the warp would
+      // block anyway, on P: V item j before PV0(j)'s P (PV1(j) then needs no
+      // V wait: this warp has observed it), and K item j+1 probed there too
+      // (k_seen), so that PV0(j) -> S0(j+1) runs with no wait between.
       bool ok = warp_wait_bar(bar(C::kBarQ), 0, wc);
+      bool k_seen = false;  // K item of the next S0 already observed
       for (int j = 0; ok && j <= n_kv; ++j) {
         if (j < n_kv && (j <= last0 || !pair)) {
           // S0(j); unpaired, K item j also serves S1(j) and is waited for here
           const int u = item_of(0, j);
-          if (!(ok = wait_k(u))) break;
+          if (k_seen) {
+            tc_fence_after();
+          } else if (!(ok = wait_k(u))) {
+            break;
+          }
+          k_seen = false;
           if (j <= last0) issue_s(0, u % C::kKStages);
           if (pair && u + C::kKStages < n_items) mma_commit_elect(bar(C::kBarKEmpty + u % C::kKStages));
         }
         if (j >= 1 && j - 1 <= last1) {
           // PV1(j-1): the tensor cores work on it while softmax 0 handles S0(j)
           const int jp = j - 1, u = item_of(1, jp);
-          ok = issue_pv(1, jp, u, split1 && jp == 0);
+          // unpaired: PV0(jp) observed V item jp unless jp > last0
+          ok = issue_pv(1, jp, u, split1 && jp == 0, pair || jp > last0);
           if (!ok) break;
           if (jp == last1) mma_commit_elect(bar(C::kBarOFinal + 1));
           // unpaired: PV1 is V_jp's last reader; paired: its only one
@@ -640,7 +657,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!pair && j + C::kKStages < n_kv) mma_commit_elect(bar(C::kBarKEmpty + j % C::kKStages));
           if (j <= last0) {
             const int u = item_of(0, j);
-            ok = issue_pv(0, j, u, split0 && j == 0);
+            if (!pair) {
+              // V item j, then a poll of K item j+1, before PV0(j)'s P wait
+              if (!(ok = warp_wait_bar(bar(C::kBarVFull + u % C::kVStages),
+                                       static_cast<uint32_t>((u / C::kVStages) & 1), wc)))
+                break;
+              if (j + 1 < n_kv)
+                k_seen = __all_sync(0xffffffffu, mbar_test_wait(bar(C::kBarKFull + (j + 1) % C::kKStages),
+                                                                static_cast<uint32_t>(((j + 1) / C::kKStages) & 1)));
+            }
+            ok = issue_pv(0, j, u, split0 && j == 0, pair);
             if (!ok) break;
             if (j == last0) mma_commit_elect(bar(C::kBarOFinal + 0));
             if ((pair || j > last1) && u + C::kVStages < n_items) mma_commit_elect(bar(C::kBarVEmpty + u % C::kVStages));

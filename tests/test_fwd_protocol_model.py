@@ -5,7 +5,9 @@ fa_fwd_kernel.cuh), not its arithmetic:
   * the loader warp: Q once, then for every ring item u the K tile and the V tile,
     each into stage u % S after the stage's previous item has been released;
   * the MMA warp, in the order S0(j), PV1(j-1), S1(j), PV0(j), with the commits
-    that release K/V stages, publish S_i and mark the last PV_i;
+    that release K/V stages, publish S_i and mark the last PV_i; each PV waits
+    for V before P, and unpaired the warp waits for V item j and polls K item
+    j+1 before PV0(j)'s P wait, then skips the waits those already satisfied;
   * two softmax warpgroups of four warps, each warp arriving on the two halves of
     P_i (the kernel's barriers count 128 thread arrivals; here, 4 warp arrivals).
 Items are one key tile shared by both query tiles (unpaired), or, paired (packed
@@ -13,7 +15,8 @@ heads with split-KV), alternating tile 0 / tile 1 items while both have tiles.
 
 Checked at every step: a waiter is never more than one phase behind the barrier
 it polls (a parity wait would misread it); a stage is reloaded only after every
-MMA reading its previous item has completed; an MMA reads the item it expects;
+MMA reading its previous item has completed; an MMA reads the item it expects,
+and only after the MMA warp itself has seen that item's full barrier complete;
 S_i(j) is issued only after PV_i(j-1) and after all four warps read S_i(j-1);
 PV reads P only once all four warps wrote it; and the run ends (no deadlock).
 Completions (TMA, commits) arrive at random times, commits in issue order.
@@ -96,44 +99,54 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
     def mma_warp():
         while not ready("Q", 0):
             yield
+        seen = set()  # (kind, item) whose full barrier this warp has seen complete
+
+        def observe(kind, u):
+            ok = ready(f"{kind}F{u % stages}", u // stages)
+            if ok:
+                seen.add((kind, u))
+            return ok
 
         def wait_k(u):
-            while not ready(f"KF{u % stages}", u // stages):
+            while not observe("K", u):
                 yield
 
         def issue_s(i, j):
             u = item_of(i, j)
             s = u % stages
-            if slot["K"][s] != u or not landed["K"][s]:
-                raise ProtocolError(f"S{i}({j}) reads K stage {s} without item {u}")
+            if slot["K"][s] != u or not landed["K"][s] or ("K", u) not in seen:
+                raise ProtocolError(f"S{i}({j}) reads K stage {s} without having seen item {u} land")
             if j > 0 and ((i, j - 1) not in pv_issued or not s_read.get((i, j - 1))):
                 raise ProtocolError(f"S{i}({j}) overwrites S/P of tile {j - 1} too early")
             for _ in range(8):
                 mma("K", u)
             commit(f"SF{i}")
 
-        def issue_pv(i, j, split):
+        def issue_pv(i, j, split, need_v):
             u = item_of(i, j)
             s = u % stages
+            if need_v:  # V first, then the halves of P
+                while not observe("V", u):
+                    yield
             for h in range(2):
                 while not ready(f"PF{i}{h}", j):
                     yield
-                if h == 0:
-                    while not ready(f"VF{s}", u // stages):
-                        yield
                 if not p_written.get((i, j, h)):
                     raise ProtocolError(f"PV{i}({j}) half {h} before P was written")
-                if slot["V"][s] != u or not landed["V"][s]:
-                    raise ProtocolError(f"PV{i}({j}) reads V stage {s} without item {u}")
+                if slot["V"][s] != u or not landed["V"][s] or ("V", u) not in seen:
+                    raise ProtocolError(f"PV{i}({j}) reads V stage {s} without having seen item {u} land")
                 for _ in range(8 if split else 4):
                     mma("V", u)
                 yield
             pv_issued.add((i, j))
 
+        k_seen = False  # unpaired: K item j+1 polled ready before PV0(j)'s P wait
         for j in range(n_kv + 1):
             if j < n_kv and (j <= last0 or not pair):
                 u = item_of(0, j)
-                yield from wait_k(u)
+                if not k_seen:
+                    yield from wait_k(u)
+                k_seen = False
                 if j <= last0:
                     issue_s(0, j)
                 if pair and u + stages < n_items:
@@ -141,7 +154,11 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
                 yield
             if 1 <= j and j - 1 <= last1:
                 u = item_of(1, j - 1)
-                yield from issue_pv(1, j - 1, split1 and j == 1)
+                # unpaired: PV0(j-1) observed V item j-1 unless j-1 > last0
+                need_v = pair or j - 1 > last0 or plant == "always_skip_v"
+                if plant == "always_skip_v" and not pair:
+                    need_v = False
+                yield from issue_pv(1, j - 1, split1 and j == 1, need_v)
                 if j - 1 == last1:
                     commit("OF1")
                 if u + stages < n_items:
@@ -158,7 +175,16 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
                     commit(f"KE{j % stages}")
                 if j <= last0:
                     u = item_of(0, j)
-                    yield from issue_pv(0, j, split0 and j == 0)
+                    if not pair:
+                        # V item j, then one poll of K item j+1, before the P wait
+                        while not observe("V", u):
+                            yield
+                        if j + 1 < n_kv:
+                            k_seen = observe("K", j + 1)
+                            if plant == "k_probe_stage":
+                                k_seen = True  # a poll taken as satisfied without looking
+                        yield
+                    yield from issue_pv(0, j, split0 and j == 0, pair)
                     if j == last0:
                         commit("OF0")
                     if (pair or j > last1) and u + stages < n_items and plant != "late_v_release":
@@ -239,4 +265,15 @@ def test_protocol_model_catches_planted_bugs(plant):
     with pytest.raises(ProtocolError):
         for case in _cases(600, 0):
             if case[2]:  # paired cases exercise all three plants
+                simulate(*case, plant=plant)
+
+
+@pytest.mark.parametrize("plant", ["always_skip_v", "k_probe_stage"])
+def test_protocol_model_catches_planted_unpaired_bugs(plant):
+    """Unpaired plants: PV1 skipping its V wait also where PV0 did not observe
+    that item (query tile 0 ends a tile earlier), and the K poll's result taken
+    as ready without looking."""
+    with pytest.raises(ProtocolError):
+        for case in _cases(600, 0):
+            if not case[2]:
                 simulate(*case, plant=plant)
