@@ -44,6 +44,9 @@ class _Bar:
 
 
 def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant=None):
+    # stages: K and V ring depths, (kstages, vstages), or one int for both
+    ks, vs = stages if isinstance(stages, tuple) else (stages, stages)
+    depth = {"K": ks, "V": vs}
     rng = random.Random(seed)
     n_kv = max(last0, last1) + 1
     n_items = (last0 + 1) + (last1 + 1) if pair else n_kv
@@ -56,15 +59,16 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
         return 2 * j + i if j <= last1 else last1 + 1 + j
 
     bars = {"Q": _Bar(1)}
-    for s in range(stages):
-        for name in ("KF", "KE", "VF", "VE"):
-            bars[f"{name}{s}"] = _Bar(1)
+    for kind in "KV":
+        for s in range(depth[kind]):
+            for name in ("F", "E"):
+                bars[f"{kind}{name}{s}"] = _Bar(1)
     for i in range(2):
         bars[f"SF{i}"], bars[f"OF{i}"] = _Bar(1), _Bar(1)
         for h in range(2):
             bars[f"PF{i}{h}"] = _Bar(4)
-    slot = {"K": [None] * stages, "V": [None] * stages}
-    landed = {"K": [False] * stages, "V": [False] * stages}
+    slot = {"K": [None] * ks, "V": [None] * vs}
+    landed = {"K": [False] * ks, "V": [False] * vs}
     events, mmas, done, readers = [], [], set(), {}
     s_read, p_written, pv_issued = {}, {}, set()
 
@@ -86,12 +90,13 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
         events.append(("q",))
         for u in range(n_items):
             for kind in "KV":
-                s = u % stages
-                if u >= stages:
-                    while not ready(f"{kind}E{s}", u // stages - 1):
+                n = depth[kind]
+                s = u % n
+                if u >= n:
+                    while not ready(f"{kind}E{s}", u // n - 1):
                         yield
-                    if any(m not in done for m in readers.get((kind, u - stages), [])):
-                        raise ProtocolError(f"{kind} stage {s} reloaded while item {u - stages} is read")
+                    if any(m not in done for m in readers.get((kind, u - n), [])):
+                        raise ProtocolError(f"{kind} stage {s} reloaded while item {u - n} is read")
                 slot[kind][s], landed[kind][s] = u, False
                 events.append(("tma", kind, s))
                 yield
@@ -102,7 +107,7 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
         seen = set()  # (kind, item) whose full barrier this warp has seen complete
 
         def observe(kind, u):
-            ok = ready(f"{kind}F{u % stages}", u // stages)
+            ok = ready(f"{kind}F{u % depth[kind]}", u // depth[kind])
             if ok:
                 seen.add((kind, u))
             return ok
@@ -113,7 +118,7 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
 
         def issue_s(i, j):
             u = item_of(i, j)
-            s = u % stages
+            s = u % ks
             if slot["K"][s] != u or not landed["K"][s] or ("K", u) not in seen:
                 raise ProtocolError(f"S{i}({j}) reads K stage {s} without having seen item {u} land")
             if j > 0 and ((i, j - 1) not in pv_issued or not s_read.get((i, j - 1))):
@@ -124,7 +129,7 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
 
         def issue_pv(i, j, split, need_v):
             u = item_of(i, j)
-            s = u % stages
+            s = u % vs
             if need_v:  # V first, then the halves of P
                 while not observe("V", u):
                     yield
@@ -149,8 +154,8 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
                 k_seen = False
                 if j <= last0:
                     issue_s(0, j)
-                if pair and u + stages < n_items:
-                    commit(f"KE{u % stages}")
+                if pair and u + ks < n_items:
+                    commit(f"KE{u % ks}")
                 yield
             if 1 <= j and j - 1 <= last1:
                 u = item_of(1, j - 1)
@@ -161,18 +166,18 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
                 yield from issue_pv(1, j - 1, split1 and j == 1, need_v)
                 if j - 1 == last1:
                     commit("OF1")
-                if u + stages < n_items:
-                    commit(f"VE{u % stages}")
+                if u + vs < n_items:
+                    commit(f"VE{u % vs}")
             if j < n_kv:
                 if j <= last1:
                     u = item_of(1, j)
                     if pair and plant != "skip_k_wait":
                         yield from wait_k(u)
                     issue_s(1, j)
-                    if pair and u + stages < n_items:
-                        commit(f"KE{u % stages}")
-                if not pair and j + stages < n_kv:
-                    commit(f"KE{j % stages}")
+                    if pair and u + ks < n_items:
+                        commit(f"KE{u % ks}")
+                if not pair and j + ks < n_kv:
+                    commit(f"KE{j % ks}")
                 if j <= last0:
                     u = item_of(0, j)
                     if not pair:
@@ -187,10 +192,10 @@ def simulate(last0, last1, pair, stages, seed, split0=False, split1=False, plant
                     yield from issue_pv(0, j, split0 and j == 0, pair)
                     if j == last0:
                         commit("OF0")
-                    if (pair or j > last1) and u + stages < n_items and plant != "late_v_release":
-                        commit(f"VE{u % stages}")
-                    elif plant == "late_v_release" and j > last1 and u + stages < n_items:
-                        commit(f"VE{u % stages}")
+                    if (pair or j > last1) and u + vs < n_items and plant != "late_v_release":
+                        commit(f"VE{u % vs}")
+                    elif plant == "late_v_release" and j > last1 and u + vs < n_items:
+                        commit(f"VE{u % vs}")
             yield
 
     def softmax_warp(i, w):
@@ -244,7 +249,8 @@ def _cases(n, seed0):
     out = []
     for seed in range(seed0, seed0 + n):
         r = random.Random(seed)
-        stages = r.choice([2, 4])  # the kernel's K/V stage counts at D = 128 and 64
+        # K / V ring depths: the kernel's at D = 128 and D = 64, and asymmetric rings
+        stages = r.choice([(2, 2), (2, 3), (3, 2), (4, 4), (6, 6)])
         if r.random() < 0.5:
             t = r.randint(1, 8)  # tiles per key range
             out.append((t - 1, r.choice([-1, r.randint(0, t - 1), t - 1]), True, stages, seed, False, False))
