@@ -158,12 +158,34 @@ def _dtype_code(t) -> int:
     raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
 
 
-def _check_cuda(**tensors):
+def _check_cuda(device=None, **tensors):
+    """Every tensor is a contiguous CUDA tensor, on ``device`` when given (the
+    library receives raw pointers: a host pointer or another GPU's memory
+    would reach the kernels unchecked)."""
     for name, t in tensors.items():
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+        if device is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}; every tensor must be on {device}")
+
+
+def _check_like(name, t, shape, dtype):
+    """A caller-provided output has exactly the shape and dtype the kernels write."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {list(shape)}, got {t.dtype} {list(t.shape)}")
+
+
+def _check_qkv4(q, k, v):
+    """q [B, Nq, Hq, D] and k, v [B, Nk, Hkv, D] of one 16-bit dtype."""
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q must be [B, Nq, Hq, D] and k, v [B, Nk, Hkv, D]")
+    if k.shape[0] != q.shape[0] or k.shape[3] != q.shape[3]:
+        raise ValueError("q and k/v disagree on batch or head dimension")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    _dtype_code(q)
 
 
 def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, **debug) -> None:
@@ -182,10 +204,10 @@ def fwd_into(q, k, v, o, lse, scale: float | None = None, causal: bool = False, 
         raise ValueError("q and k/v disagree on batch or head dimension")
     if tuple(lse.shape) != (B, Hq, Nq) or lse.dtype != torch.float32:
         raise ValueError("lse must be float32 [B, Hq, Nq]")
-    _check_cuda(q=q, k=k, v=v, o=o, lse=lse)
     if k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
         raise TypeError("q, k, v and o must share one dtype")
     code = _dtype_code(q)
+    _check_cuda(q.device, q=q, k=k, v=v, o=o, lse=lse)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream(q.device).cuda_stream
@@ -230,13 +252,16 @@ def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, scale: fl
     if cu_seqlens_q.dim() != 1 or cu_seqlens_k.shape != cu_seqlens_q.shape:
         raise ValueError("cu_seqlens_q and cu_seqlens_k must be 1-D with B+1 entries")
     B = cu_seqlens_q.numel() - 1
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    _dtype_code(q)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
-    _check_cuda(q=q, k=k, v=v, o=o, lse=lse, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k)
-    if k.dtype != q.dtype or v.dtype != q.dtype or o.dtype != q.dtype:
-        raise TypeError("q, k, v and o must share one dtype")
+    _check_like("o", o, q.shape, q.dtype)
+    _check_like("lse", lse, (Hq, total_q), torch.float32)
+    _check_cuda(q.device, q=q, k=k, v=v, o=o, lse=lse, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream(q.device).cuda_stream
@@ -272,11 +297,16 @@ def fwd_splitkv(q, k, v, scale: float | None = None, causal: bool = False, num_s
     """
     import torch
 
+    _check_qkv4(q, k, v)
     B, Nq, Hq, D = q.shape
     _, Nk, Hkv, _ = k.shape
-    _check_cuda(q=q, k=k, v=v)
-    if k.dtype != q.dtype or v.dtype != q.dtype:
-        raise TypeError("q, k and v must share one dtype")
+    if o is not None:
+        _check_like("o", o, q.shape, q.dtype)
+    if lse is not None:
+        _check_like("lse", lse, (B, Hq, Nq), torch.float32)
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    _check_cuda(q.device, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     with torch.cuda.device(q.device):
@@ -287,7 +317,7 @@ def fwd_splitkv(q, k, v, scale: float | None = None, causal: bool = False, num_s
             o = torch.empty_like(q)
         if lse is None:
             lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-        _check_cuda(o=o, lse=lse)
+        _check_cuda(q.device, o=o, lse=lse, workspace=workspace)
         stream = torch.cuda.current_stream(q.device).cuda_stream
         st = load_library().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                                            B, Nq, Nk, Hq, Hkv, D, ctypes.c_float(float(scale)), int(bool(causal)),
@@ -310,9 +340,12 @@ def fwd_splitkv_noalloc(q, k, v, o, lse, scale: float | None = None, causal: boo
     results raise FaError(FA_ERR_UNSUPPORTED)."""
     import torch
 
+    _check_qkv4(q, k, v)
     B, Nq, Hq, D = q.shape
     _, Nk, Hkv, _ = k.shape
-    _check_cuda(q=q, k=k, v=v, o=o, lse=lse)
+    _check_like("o", o, q.shape, q.dtype)
+    _check_like("lse", lse, (B, Hq, Nq), torch.float32)
+    _check_cuda(q.device, q=q, k=k, v=v, o=o, lse=lse)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream(q.device).cuda_stream
@@ -369,7 +402,7 @@ def bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False,
         need = bwd_workspace_size(B, Nq, Hq)
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-        _check_cuda(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace)
+        _check_cuda(q.device, q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace)
         stream = torch.cuda.current_stream(q.device).cuda_stream
         args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
@@ -409,14 +442,20 @@ def bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: 
     B = cu_seqlens_q.numel() - 1
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    _dtype_code(q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(k) if dv is None else dv
+    _check_like("dq", dq, q.shape, q.dtype)
+    _check_like("dk", dk, k.shape, q.dtype)
+    _check_like("dv", dv, k.shape, q.dtype)
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
     with torch.cuda.device(q.device):
         need = bwd_workspace_size(B, max_seqlen_q, Hq)
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-        _check_cuda(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace,
+        _check_cuda(q.device, q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, workspace=workspace,
                     cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k)
         stream = torch.cuda.current_stream(q.device).cuda_stream
         st = load_library().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
